@@ -1,0 +1,366 @@
+"""Benchmark of the hybrid compressed attention core on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch of synthetic input: for the
+default CSA prefill workload (B=1, S=8192, 64 heads, head_dim 512, m=4, top-512,
+window 128) that is compress(kv) + compress(kI) + indexer/top-k + sparse attention.
+``value`` is whole-job tokens/s with inputs resident in HBM (device time, CUDA events,
+max over ranks); ``e2e`` is the same metric through the layer entry point with pinned
+host inputs copied in and the output copied back every step.  With N > 1 every rank
+runs its own batch (independent sequences, no data-path collective): weak scaling.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of query rows.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "CSA/HCA layer prefill tokens/s and decode µs/step on 1 B200; % of roofline"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def attn_keys_per_query(w, q_index):
+    """Keys each query attends: window tokens plus min(topk, visible) pool entries."""
+    t = q_index.reshape(-1).astype(np.int64)
+    win = np.minimum(w.n_win, t + 1) if w.n_win > 0 else np.zeros_like(t)
+    vis = np.minimum((t + 1) // w.m, w.P_cap)
+    pool = np.minimum(vis, w.topk) if w.kind != "hca" else vis
+    return win + pool
+
+
+def attn_flops(w, q_index):
+    """Algorithmic FLOPs of one attention launch: H x keys x (D for QK^T + dv for PV) x 2."""
+    return float(attn_keys_per_query(w, q_index).sum()) * w.H * (w.D + w.dv) * 2.0
+
+
+def attn_bytes(w, q_index):
+    """Algorithmic HBM bytes of one attention launch: q, out, gathered K=V rows, idx."""
+    e = 2 if w.dtype == "bf16" else 4
+    nq = w.B * w.Sq
+    keys = float(attn_keys_per_query(w, q_index).sum())
+    return nq * w.H * (w.D + w.dv) * e + keys * w.D * e + (nq * w.topk * 4 if w.topk else 0)
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for (ts, s) in self.samples if t0 <= ts <= t1] or [s for _, s in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_rate(w, budget_s: float, host=None):
+    """Time the fp64 oracle on a bounded, time-limited sample of the workload's query rows.
+
+    Returns (tokens_per_s, rows_done, seconds, description).  The sample starts with the
+    compression of the whole sequence (for prefill workloads) and then runs indexer + top-k
+    + attention row by row over a strided sample of query rows until `budget_s` elapses.
+    """
+    from oracle import dsv4_oracle as O
+    if host is None:
+        host = synth.make_inputs(w) if w.kind != "decode" else None
+    t0 = time.perf_counter()
+    if w.kind == "decode":
+        sp = synth.cache_specs(w)
+        specs = synth.tensor_specs(w)
+        qi, qpos = synth.positions(w)
+        done = 0
+        for b in range(w.B):
+            pool = sp["pool"].rows(b * w.P_cap, (b + 1) * w.P_cap)[None]
+            poolI = sp["poolI"].rows(b * w.P_cap, (b + 1) * w.P_cap)[None]
+            win = sp["win"].rows(b * w.win_ring, (b + 1) * w.win_ring)[None]
+            q = specs["q"].rows(b, b + 1).reshape(1, 1, w.H, w.D)
+            qI = specs["qI"].rows(b, b + 1).reshape(1, 1, w.nI, w.cI)
+            wI = specs["wI"].rows(b, b + 1).reshape(1, 1, w.nI)
+            sink = specs["sink"].full()
+            idx = O.indexer_topk(qI, wI, poolI, qi[b:b + 1], m=w.m, topk=w.topk, P_cap=w.P_cap)
+            O.sparse_mqa_attention(q, win, pool, idx, sink, qpos[b:b + 1], qi[b:b + 1], n_win=w.n_win, m=w.m,
+                                   scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rope_q=True,
+                                   rotate_out=w.rotate_out, win_ring=w.win_ring, P_cap=w.P_cap)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return done / dt, done, dt, f"{done} of {w.B} decode sequences (indexer + top-k + attention)"
+    kw = dict(m=w.m, n_win=w.n_win, scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rotate_out=w.rotate_out)
+    pool = O.compress(host["kv"], host.get("z"), host.get("bias"), host["pos"], m=w.m, overlap=w.overlap,
+                      apply_rope=True, R=w.R, theta=w.theta)
+    kv_rot = O.rope_rotate(host["kv"], host["pos"], w.R, w.theta)
+    poolI = O.compress(host["kI"], host.get("zI"), host.get("biasI"), host["pos"], m=w.m,
+                       overlap=w.overlap, apply_rope=False) if w.nI > 0 else None
+    t_comp = time.perf_counter() - t0
+    order = np.random.default_rng(0).permutation(w.S)
+    done = 0
+    t1 = time.perf_counter()
+    qi = np.tile(np.arange(w.S), (w.B, 1))
+    for s in order:
+        rows = [(0, int(s))]
+        idx = O.indexer_topk(host["qI"], host["wI"], poolI, qi, m=w.m, topk=w.topk, rows=rows) \
+            if w.nI > 0 else None
+        O.sparse_mqa_attention(host["q"], kv_rot, pool, idx, host["sink"], host["pos"], qi, rope_q=True,
+                               rows=rows, **{k: v for k, v in kw.items()})
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    t_rows = time.perf_counter() - t1
+    per_row = t_rows / max(done, 1)
+    total = t_comp + per_row * w.S * w.B
+    return (w.S * w.B) / total, done, t_comp + t_rows, (
+        f"compression of all {w.S} tokens ({t_comp:.2f} s) + {done} random query rows "
+        f"({per_row * 1e3:.1f} ms/row), extrapolated to {w.S} rows")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    host = synth.make_inputs(w) if w.kind != "decode" else None
+    per_step = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        rate, rows, secs, desc = cpu_oracle_rate(w, args.ref_budget, host)
+        if i >= args.warmup:
+            per_step.append(rate)
+    if w.kind == "decode":
+        value = 1e6 / float(np.mean(per_step)) * w.B  # us per step of all B sequences
+        unit = "us/step"
+    else:
+        value = float(np.mean(per_step))
+        unit = "tokens/s"
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": unit == "tokens/s",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    c = {"workload": w.name, "B": w.B, "S": w.S, "Sq": w.Sq, "H": w.H, "head_dim": w.D, "rope_dim": w.R,
+         "dv": w.dv, "sliding_window": w.n_win, "m": w.m, "overlap": w.overlap, "pool_cap": w.P_cap}
+    if w.nI:
+        c.update({"index_n_heads": w.nI, "index_head_dim": w.cI, "index_topk": w.topk})
+    c["l2"] = "inputs larger than L2 (q and out are each > 126 MB)" if w.B * w.Sq * w.H * w.D * 2 > (126 << 20) \
+        else "L2 flushed between steps"
+    return c
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="csa_prefill_bf16", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from sparse_long_context_csa_b200 import abi, harness
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    abi.load()
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    o = harness.make_outputs(w, params)
+    stream = torch.cuda.current_stream()
+    q_index = host["q_index"]
+
+    def step(ev_pair=None):
+        harness.step_parts(w, params, x, o, stream, attn_events=ev_pair)
+
+    # warm-up (also starts the clock sampler and lets it settle)
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t_w = time.time()
+    while time.time() - t_w < 1.0:  # keep the GPU busy while nvidia-smi starts sampling
+        step()
+        torch.cuda.synchronize()
+
+    # timed region: K steps, device time, attention kernel timed separately
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = abi.dsv4_launch_count()
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    n1 = abi.dsv4_launch_count()
+    barrier()
+    ms = max_over_ranks(start.elapsed_time(end))
+    attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+    clocks = sampler.summary(wall0, wall1)
+
+    # end to end through the layer entry point: pinned host inputs in, output back
+    host_t = harness.to_device(w, host, device=None, pin=True)
+    out_host = torch.empty(o["out"].shape, dtype=o["out"].dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_t.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for k, t in host_t.items():
+            x[k].copy_(t, non_blocking=True)
+        harness.step(w, params, x, o, stream)
+        out_host.copy_(o["out"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    sampler.stop()
+
+    tokens = w.B * w.Sq
+    ms_step = ms / args.steps
+    if w.kind == "decode":
+        value, unit, hib = ms_step * 1e3, "us/step", False
+        e2e_val = e2e_ms * 1e3
+    else:
+        value, unit, hib = world * tokens * args.steps / (ms / 1e3), "tokens/s", True
+        e2e_val = world * tokens / (e2e_ms / 1e3)
+
+    peaks, peak_src = _peaks()
+    if w.kind == "decode":
+        achieved = attn_bytes(w, q_index) / (attn_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "sparse attention", "peak_source": f"{peak_src} hbm_gbs"}
+    else:
+        achieved = attn_flops(w, q_index) / (attn_ms / 1e3) / 1e12
+        pk = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
+                "traffic": None, "kernel": "sparse attention",
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+    roof["kernel_ms"] = attn_ms
+
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": hib, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1)/sqrt(d) inputs, no weights)",
+            "config": config_of(w), "parallelism": f"replicas x{world} (independent sequences)",
+            "gpu_launches": int(n1 - n0), "clocks": clocks, "roofline": roof,
+            "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, rows, secs, desc = cpu_oracle_rate(w, args.cpu_budget, host)
+        cv = (1e6 / rate * w.B) if w.kind == "decode" else rate
+        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                                "sample": desc, "seconds": round(secs, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

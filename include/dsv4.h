@@ -1,0 +1,194 @@
+/*
+ * dsv4.h — C ABI of libdsv4, the DeepSeek-V4 hybrid compressed attention core
+ * (CSA / HCA, and the token-level DSA variant) on NVIDIA B200 (sm_100a).
+ *
+ * Method sources (HF Transformers model docs):
+ *   [V4]  "DeepSeek-V4" doc: section "Architecture (paper §2)" → "Hybrid attention
+ *         (§2.3)" (CSA / HCA items, shared K=V MQA, partial RoPE and the -i output
+ *         rotation of eq. 26, per-head sink of eq. 27, sliding-window K=V branch),
+ *         "Attention mask layout" (visibility rules, -1 sentinels), "Cache layers",
+ *         and the DeepseekV4Config parameters (sliding_window, compress_rates,
+ *         compress_rope_theta, index_n_heads, index_head_dim, index_topk).
+ *   [V32] "DeepSeek-V3.2" doc: section "DeepSeek Sparse Attention (DSA)"
+ *         (Lightning Indexer, fine-grained top-k token selection).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; they must be
+ *     16-byte aligned and the tensors contiguous, row-major, in the shapes given.
+ *     "T" is the activation dtype named by params->dtype (float32 or bfloat16).
+ *   - The library allocates no memory and keeps no state between calls.  Scratch
+ *     space is the caller's `workspace` of at least dsv4_workspace_bytes(params).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are validated on the host before any launch;
+ *     an invalid call returns a non-zero dsv4_status and enqueues nothing.
+ *   - No entry point aborts, traps or synchronises the device.  DSV4_ERR_CUDA
+ *     means a launch was refused by the runtime (cudaGetLastError).
+ *
+ * Index conventions
+ *   - Cache index t of a query decides visibility; RoPE positions (pos, qpos)
+ *     only feed the rotations, so shifting every position leaves outputs unchanged.
+ *   - A query at cache index t sees pool entries w < min((t+1)/m, P_cap) ([V4]
+ *     "Attention mask layout": an entry is visible once its window has closed) and
+ *     the window tokens (t - n_win, t] ∩ [0, t].
+ */
+#ifndef DSV4_H_
+#define DSV4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSV4_OK = 0,
+  DSV4_ERR_ARG = 1,          /* null pointer where one is required, or bad flag value */
+  DSV4_ERR_SHAPE = 2,        /* sizes inconsistent or outside what the kernels support */
+  DSV4_ERR_ALIGN = 3,        /* a tensor pointer is not 16-byte aligned */
+  DSV4_ERR_DTYPE = 4,        /* unknown params->dtype */
+  DSV4_ERR_CUDA = 5,         /* the CUDA runtime refused a launch or query */
+  DSV4_ERR_DEVICE_CHECK = 6, /* reserved: a device-side check word reported a bad index */
+  DSV4_ERR_WORKSPACE = 7     /* workspace missing or smaller than dsv4_workspace_bytes() */
+} dsv4_status;
+
+typedef enum { DSV4_F32 = 0, DSV4_BF16 = 1 } dsv4_dtype;
+
+/* Sizes of one call.  Nothing has a hidden default: the caller sets every field. */
+typedef struct dsv4_params {
+  int32_t B;          /* sequences in the batch */
+  int32_t S;          /* tokens per sequence in kv / kI / x (prefill and compress) */
+  int32_t Sq;         /* query tokens per sequence */
+  int32_t H;          /* query heads (num_attention_heads); one shared K=V head */
+  int32_t D;          /* head_dim: width of q rows and K=V rows */
+  int32_t R;          /* trailing rotary channels (qk_rope_head_dim), even, <= D */
+  int32_t dv;         /* value width: the first dv channels of each K=V row */
+  int32_t n_win;      /* sliding_window (0 = no window branch) */
+  int32_t win_ring;   /* 0: window rows addressed by cache index in [B,S,D];
+                         >0: ring buffer [B,win_ring,D], token j in slot j % win_ring
+                         (requires win_ring >= n_win) */
+  int32_t m;          /* compression rate (compress_rates: 4 CSA, 128 HCA, 1 DSA) */
+  int32_t overlap;    /* 1: entry w pools tokens [(w-1)m,(w+1)m) (CSA); 0: [wm,(w+1)m) */
+  int32_t P_cap;      /* pool capacity: entries per sequence in pool / poolI buffers */
+  int32_t nI;         /* index_n_heads */
+  int32_t cI;         /* index_head_dim */
+  int32_t topk;       /* index_topk */
+  float scale;        /* softmax scale applied to q.k (e.g. 1/sqrt(D)) */
+  float rope_theta;   /* RoPE base (compress_rope_theta for CSA/HCA, rope_theta for DSA) */
+  int32_t rope_q;     /* 1: rotate q at qpos inside the attention; 0: q already rotated */
+  int32_t rotate_out; /* 1: rotate the output rope slice by -qpos (eq. 26); needs dv == D */
+  int32_t dtype;      /* dsv4_dtype of every activation tensor "T" */
+} dsv4_params;
+
+/*
+ * KV compressor ([V4] "Hybrid attention (§2.3)", CSA item: low-compression pool with
+ * overlapping windows; HCA item: high-compression pool, non-overlapping windows;
+ * "Cache layers": the indexer keys get their own pool at index_head_dim).
+ *
+ * Pools token rows x into entries: for each entry w < S/m and channel d,
+ *   pool[w,d] = sum_{j in J_w} alpha_j[d] x[j,d],
+ *   alpha_.[d] = softmax over J_w of (z[j,d] + bias[slot(j),d]),
+ * with J_w = [(w-1)m, (w+1)m) ∩ [0,S) and slot(j) = j-(w-1)m when overlap, else
+ * J_w = [wm,(w+1)m), slot(j) = j-wm.  With apply_rope, the entry's trailing R channels
+ * are rotated (interleaved pairs, base rope_theta) at pos[b, w*m].
+ *
+ *   c      channels per row (D for the K=V stream, cI for the indexer-key stream)
+ *   x      [B,S,c] T          token rows (not rotated)
+ *   z      [B,S,c] T or NULL  per-token compressor logits (NULL = 0)
+ *   bias   [2m or m, c] f32 or NULL   per-slot bias (NULL = 0)
+ *   pos    [B,S] int64        RoPE positions (required when apply_rope)
+ *   pool   [B,P_cap,c] T      out: entries 0 .. S/m-1 are written (S/m <= P_cap)
+ *   x_rot  [B,S,c] T or NULL  out: x rotated at pos (the window keys); needs apply_rope
+ */
+dsv4_status dsv4_compress_kv(const dsv4_params* params, int32_t c, const void* x, const void* z,
+                             const float* bias, const int64_t* pos, int32_t apply_rope,
+                             void* pool, void* x_rot, void* stream);
+
+/*
+ * Lightning Indexer + top-k ([V4] CSA item, eqs. 13-17 and index_topk (eq. 17);
+ * [V32] DSA items 1-2).  For each query (b,s) at cache index t = q_index[b,s] and
+ * every visible entry w < vis = min((t+1)/m, P_cap):
+ *   I[w] = sum_h wI[b,s,h] * relu(qI[b,s,h,:] . poolI[b,w,:])
+ * then keeps the min(topk, vis) entries of highest I (ties: lower w wins).
+ *
+ *   qI      [B,Sq,nI,cI] T
+ *   wI      [B,Sq,nI] f32       per-head index weights
+ *   poolI   [B,P_cap,cI] T      compressed indexer keys (no RoPE)
+ *   q_index [B,Sq] int32 or NULL  cache index of each query (NULL: q_index[b,s] = s)
+ *   idx     [B,Sq,topk] int32   out: selected entries in ASCENDING entry order, then -1
+ *   workspace, ws_bytes         >= dsv4_workspace_bytes(params)
+ */
+dsv4_status dsv4_indexer_topk(const dsv4_params* params, const void* qI, const float* wI,
+                              const void* poolI, const int32_t* q_index, int32_t* idx,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse shared-K=V MQA attention with sink ([V4] "Hybrid attention (§2.3)": one KV
+ * head read as key and value, partial RoPE, -i output rotation (eq. 26), per-head sink
+ * (eq. 27), sliding-window K=V branch concatenated with the compressor entries).
+ * For query (b,s) at cache index t and head h, the keys are the window rows of tokens
+ * (t-n_win, t] followed by the pool entries idx[b,s,:] that are >= 0; each key row k
+ * is also its value v = k[0:dv]:
+ *   l_j = scale * <q_h, k_j>,   o_h = sum_j e^{l_j} v_j / (e^{sink_h} + sum_j e^{l_j})
+ *
+ *   q       [B,Sq,H,D] T       rotated at qpos inside when rope_q (else already rotated)
+ *   kv_win  window rows, already rotated: [B,S,D] T (win_ring == 0) or [B,win_ring,D] T
+ *   pool    [B,P_cap,D] T      compressed entries, already rotated
+ *   idx     [B,Sq,topk] int32 or NULL   selected entries (-1 = empty slot); every entry
+ *                              must be visible and appear once.  NULL: every visible
+ *                              entry is attended (HCA, no indexer).
+ *   sink    [H] f32            per-head sink logits
+ *   qpos    [B,Sq] int64       RoPE position of each query (needed if rope_q/rotate_out)
+ *   q_index [B,Sq] int32 or NULL   cache index of each query (NULL: s); with
+ *                              win_ring == 0 window tokens at or past S select nothing
+ *   out     [B,Sq,H,dv] T
+ */
+dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* params, const void* q, const void* kv_win,
+                                 const void* pool, const int32_t* idx, const float* sink,
+                                 const int64_t* qpos, const int32_t* q_index, void* out,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * One CSA layer in prefill (Sq == S, query s at cache index s, RoPE position pos[b,s]):
+ * compress kv -> pool (rotated) and kv_rot (window keys), compress kI -> poolI,
+ * indexer + top-k -> idx, sparse attention -> out.  With m == 1, overlap == 0,
+ * n_win == 0 this is the token-level DSA layer of [V32].
+ *   q [B,S,H,D] T (not rotated); kv [B,S,D] T; z [B,S,D] T or NULL; bias [Lw,D] f32 or NULL
+ *   qI [B,S,nI,cI] T; wI [B,S,nI] f32; kI [B,S,cI] T; zI [B,S,cI] T or NULL;
+ *   biasI [Lw,cI] f32 or NULL; sink [H] f32; pos [B,S] int64
+ *   out [B,S,H,dv] T; pool [B,P_cap,D] T; poolI [B,P_cap,cI] T; kv_rot [B,S,D] T
+ *   idx [B,S,topk] int32 or NULL (NULL: kept in the workspace)
+ */
+dsv4_status dsv4_csa_layer(const dsv4_params* params, const void* q, const void* kv,
+                           const void* z, const float* bias, const void* qI, const float* wI,
+                           const void* kI, const void* zI, const float* biasI, const float* sink,
+                           const int64_t* pos, void* out, void* pool, void* poolI, void* kv_rot,
+                           int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * One HCA layer in prefill: compress kv -> pool (non-overlapping, rotated) and kv_rot,
+ * then attention over every visible entry plus the window.  Requires overlap == 0.
+ */
+dsv4_status dsv4_hca_layer(const dsv4_params* params, const void* q, const void* kv,
+                           const void* z, const float* bias, const float* sink,
+                           const int64_t* pos, void* out, void* pool, void* kv_rot,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace any entry point needs for these params (a pure function of them). */
+size_t dsv4_workspace_bytes(const dsv4_params* params);
+
+/* Static, NUL-terminated description of a status code. */
+const char* dsv4_status_string(dsv4_status status);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t dsv4_version(void);
+
+/* Kernels this process has enqueued through libdsv4 so far (all devices, all entry
+ * points); a monotone counter for launch accounting, read without synchronising. */
+uint64_t dsv4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSV4_H_ */

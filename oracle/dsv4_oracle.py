@@ -46,6 +46,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
+    "store_as",
     "rope_rotate",
     "pool_window",
     "compress",
@@ -63,6 +64,25 @@ __all__ = [
 
 def _f64(a):
     return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+def store_as(a, store):
+    """Round float64 values to the storage dtype the caller keeps them in.
+
+    store=None keeps float64; "f32" rounds to float32; "bf16" rounds to the nearest
+    bfloat16 (ties to even), as a cache of bf16 rows would.  Decisions taken on stored
+    values (top-k over indexer scores of a bf16 key pool) are then taken on the same
+    values the kernels read.
+    """
+    if store is None:
+        return _f64(a)
+    f = np.asarray(a, dtype=np.float32)
+    if store == "f32":
+        return f.astype(np.float64)
+    assert store == "bf16", store
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return r.view(np.float32).astype(np.float64)
 
 
 # --------------------------------------------------------------------------
@@ -252,7 +272,6 @@ def sparse_mqa_attention(q, kv_win, pool, idx, sink, qpos, q_index, *, n_win, m,
     rope_q: rotate q at qpos first.  rotate_out: rotate the output rope slice by
     -qpos (eq. 26).  Returns out [B,Sq,H,dv] (rows not computed stay 0).
     """
-    q = _f64(q)
     B, Sq, H, D = q.shape
     P = pool.shape[1] if P_cap is None else P_cap
     out = np.zeros((B, Sq, H, dv))
@@ -260,7 +279,7 @@ def sparse_mqa_attention(q, kv_win, pool, idx, sink, qpos, q_index, *, n_win, m,
         rows = [(b, s) for b in range(B) for s in range(Sq)]
     for b, s in rows:
         t = int(q_index[b, s])
-        q_t = rope_rotate(q[b, s], qpos[b, s], R, theta) if rope_q else q[b, s]
+        q_t = rope_rotate(q[b, s], qpos[b, s], R, theta) if rope_q else _f64(q[b, s])
         win = window_tokens(t, n_win)
         slots = [j % win_ring for j in win] if win_ring else win
         vis = visible_entries(t, m, P)
@@ -285,12 +304,17 @@ def sparse_mqa_attention(q, kv_win, pool, idx, sink, qpos, q_index, *, n_win, m,
 # HCA = compressor + core attention over every visible entry (no indexer).
 # --------------------------------------------------------------------------
 def csa_layer(q, kv, z, bias, qI, wI, kI, zI, biasI, sink, pos, *, m, overlap,
-              n_win, topk, scale, dv, R, theta, rotate_out, rows=None):
-    """Prefill CSA layer (Sq == S, query s sits at cache index s)."""
+              n_win, topk, scale, dv, R, theta, rotate_out, rows=None, store=None):
+    """Prefill CSA layer (Sq == S, query s sits at cache index s).
+
+    ``store`` rounds the pools and the rotated window rows to the dtype a cache keeps
+    them in before they are read again (see ``store_as``).
+    """
     B, S = kv.shape[0], kv.shape[1]
-    pool = compress(kv, z, bias, pos, m=m, overlap=overlap, apply_rope=True, R=R, theta=theta)
-    poolI = compress(kI, zI, biasI, pos, m=m, overlap=overlap, apply_rope=False)
-    kv_rot = rope_rotate(kv, pos, R, theta)
+    pool = store_as(compress(kv, z, bias, pos, m=m, overlap=overlap, apply_rope=True, R=R,
+                             theta=theta), store)
+    poolI = store_as(compress(kI, zI, biasI, pos, m=m, overlap=overlap, apply_rope=False), store)
+    kv_rot = store_as(rope_rotate(kv, pos, R, theta), store)
     q_index = np.tile(np.arange(S), (B, 1))
     idx = indexer_topk(qI, wI, poolI, q_index, m=m, topk=topk, rows=rows)
     out = sparse_mqa_attention(q, kv_rot, pool, idx, sink, pos, q_index, n_win=n_win, m=m,
@@ -300,11 +324,12 @@ def csa_layer(q, kv, z, bias, qI, wI, kI, zI, biasI, sink, pos, *, m, overlap,
 
 
 def hca_layer(q, kv, z, bias, sink, pos, *, m, n_win, scale, dv, R, theta, rotate_out,
-              rows=None):
+              rows=None, store=None):
     """Prefill HCA layer: non-overlapping pool, every visible entry attended."""
     B, S = kv.shape[0], kv.shape[1]
-    pool = compress(kv, z, bias, pos, m=m, overlap=False, apply_rope=True, R=R, theta=theta)
-    kv_rot = rope_rotate(kv, pos, R, theta)
+    pool = store_as(compress(kv, z, bias, pos, m=m, overlap=False, apply_rope=True, R=R,
+                             theta=theta), store)
+    kv_rot = store_as(rope_rotate(kv, pos, R, theta), store)
     q_index = np.tile(np.arange(S), (B, 1))
     out = sparse_mqa_attention(q, kv_rot, pool, None, sink, pos, q_index, n_win=n_win, m=m,
                                scale=scale, dv=dv, R=R, theta=theta, rope_q=True,

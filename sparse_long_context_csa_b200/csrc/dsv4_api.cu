@@ -1,0 +1,252 @@
+// C ABI of libdsv4: host-side validation, workspace layout and kernel dispatch.
+// Declarations and the full contract of each entry point are in include/dsv4.h.
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "internal.h"
+
+using namespace dsv4;
+
+namespace dsv4 {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace dsv4
+
+namespace {
+
+constexpr size_t kScoresBudget = 256ull << 20;  // fp32 score rows kept per indexer chunk
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+
+dsv4_status check_common(const dsv4_params* p) {
+  if (!p) return DSV4_ERR_ARG;
+  if (p->dtype != DSV4_F32 && p->dtype != DSV4_BF16) return DSV4_ERR_DTYPE;
+  if (p->B < 0 || p->S < 0 || p->Sq < 0 || p->H < 0 || p->D < 0) return DSV4_ERR_SHAPE;
+  if (p->m < 1 || (p->overlap != 0 && p->overlap != 1)) return DSV4_ERR_SHAPE;
+  if (p->P_cap < 0) return DSV4_ERR_SHAPE;
+  return DSV4_OK;
+}
+
+dsv4_status check_rope(const dsv4_params* p) {
+  if (p->R < 0 || (p->R & 1) || p->R > p->D) return DSV4_ERR_SHAPE;
+  if (!(p->rope_theta > 0.f)) return DSV4_ERR_SHAPE;
+  return DSV4_OK;
+}
+
+dsv4_status check_indexer(const dsv4_params* p) {
+  if (p->nI < 1 || p->nI > 64 || (64 % p->nI) != 0) return DSV4_ERR_SHAPE;
+  if (p->cI != 32 && p->cI != 64 && p->cI != 128) return DSV4_ERR_SHAPE;
+  if (p->topk < 1 || p->P_cap < 1) return DSV4_ERR_SHAPE;
+  return DSV4_OK;
+}
+
+dsv4_status check_attn(const dsv4_params* p) {
+  if (p->H < 1 || p->D < 2 || (p->D & 1) || p->D > 1024) return DSV4_ERR_SHAPE;
+  if (p->dv < 32 || p->dv > p->D || (p->dv % 32) != 0 || p->dv > 576) return DSV4_ERR_SHAPE;
+  if (p->n_win < 0 || p->win_ring < 0 || (p->win_ring > 0 && p->win_ring < p->n_win)) return DSV4_ERR_SHAPE;
+  if (p->rotate_out && p->dv != p->D) return DSV4_ERR_SHAPE;
+  if (!(p->scale == p->scale)) return DSV4_ERR_ARG;
+  if ((p->rope_q != 0 && p->rope_q != 1) || (p->rotate_out != 0 && p->rotate_out != 1)) return DSV4_ERR_ARG;
+  return check_rope(p);
+}
+
+size_t scores_bytes(const dsv4_params* p) {
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  if (rows == 0 || p->P_cap == 0 || p->nI < 1 || p->topk < 1) return 0;  // no indexer
+  int64_t r = indexer_rows_per_chunk(rows, p->P_cap, kScoresBudget);
+  if (r < 1) r = 1;
+  return (size_t)r * p->P_cap * sizeof(float);
+}
+
+// idx kept in the workspace by dsv4_csa_layer (a prefill call: Sq == S).
+size_t layer_idx_bytes(const dsv4_params* p) {
+  if (p->Sq != p->S || p->nI < 1 || p->topk < 1) return 0;
+  return (size_t)p->B * p->S * p->topk * sizeof(int32_t);
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+dsv4_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return DSV4_OK;
+  if (e == cudaErrorNotSupported) return DSV4_ERR_SHAPE;
+  return DSV4_ERR_CUDA;
+}
+
+dsv4_status run_compress(const dsv4_params* p, int c, const void* x, const void* z, const float* bias,
+                         const int64_t* pos, int apply_rope, void* pool, void* x_rot, void* stream) {
+  if (c < 2 || (c & 1)) return DSV4_ERR_SHAPE;
+  if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
+  if (!ok_ptr(x) || !ok_ptr(pool)) return x && pool ? DSV4_ERR_ALIGN : DSV4_ERR_ARG;
+  if ((z && !aligned16(z)) || (bias && !aligned16(bias)) || (x_rot && !aligned16(x_rot))) return DSV4_ERR_ALIGN;
+  if (apply_rope != 0 && apply_rope != 1) return DSV4_ERR_ARG;
+  if (apply_rope) {
+    if (p->R < 0 || (p->R & 1) || p->R > c || !(p->rope_theta > 0.f)) return DSV4_ERR_SHAPE;
+    if (!pos) return DSV4_ERR_ARG;
+    if (!aligned16(pos)) return DSV4_ERR_ALIGN;
+  } else if (x_rot) {
+    return DSV4_ERR_ARG;  // the rotated copy only exists with RoPE
+  }
+  CompressArgs a{};
+  a.B = p->B; a.S = p->S; a.c = c; a.m = p->m; a.overlap = p->overlap; a.P_cap = p->P_cap;
+  a.R = apply_rope ? p->R : 0; a.apply_rope = apply_rope; a.theta = p->rope_theta;
+  a.x = x; a.z = z; a.bias = bias; a.pos = pos; a.pool = pool; a.x_rot = x_rot;
+  return from_cuda(launch_compress(a, p->dtype, as_stream(stream)));
+}
+
+dsv4_status run_indexer(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
+                        const int32_t* q_index, int32_t* idx, void* scores, size_t scores_cap, void* stream) {
+  IndexerArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.nI = p->nI; a.cI = p->cI; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk;
+  a.qI = qI; a.wI = wI; a.poolI = poolI; a.q_index = q_index; a.idx = idx;
+  a.scores = static_cast<float*>(scores);
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  a.rows_per_chunk = indexer_rows_per_chunk(rows, p->P_cap, scores_cap < kScoresBudget ? scores_cap : kScoresBudget);
+  if (rows == 0) return DSV4_OK;
+  if (a.rows_per_chunk < 1) return DSV4_ERR_WORKSPACE;
+  return from_cuda(launch_indexer_topk(a, p->dtype, as_stream(stream)));
+}
+
+dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
+                     const int32_t* idx, const float* sink, const int64_t* qpos, const int32_t* q_index,
+                     void* out, void* stream) {
+  AttnArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.H = p->H; a.D = p->D; a.R = p->R; a.dv = p->dv; a.n_win = p->n_win;
+  a.win_ring = p->win_ring; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk; a.rope_q = p->rope_q;
+  a.rotate_out = p->rotate_out; a.kv_rows = p->S; a.scale = p->scale; a.theta = p->rope_theta;
+  a.q = q; a.kv_win = kv_win; a.pool = pool; a.idx = idx; a.sink = sink; a.qpos = qpos; a.q_index = q_index;
+  a.out = out;
+  if ((int64_t)p->B * p->Sq == 0) return DSV4_OK;
+  if (attn_tc_supported(a, p->dtype)) return from_cuda(launch_attn_tc(a, as_stream(stream)));
+  return from_cuda(launch_attn_simt(a, p->dtype, as_stream(stream)));
+}
+
+dsv4_status check_attn_ptrs(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
+                            const int32_t* idx, const float* sink, const int64_t* qpos, const int32_t* q_index,
+                            const void* out) {
+  if (!q || !sink || !out) return DSV4_ERR_ARG;
+  if (p->n_win > 0 && !kv_win) return DSV4_ERR_ARG;
+  if (!pool && (idx || p->P_cap > 0)) return DSV4_ERR_ARG;
+  if ((p->rope_q || p->rotate_out) && !qpos) return DSV4_ERR_ARG;
+  if (idx && p->topk < 1) return DSV4_ERR_SHAPE;
+  if (!q_index && p->Sq > p->S && p->n_win > 0 && p->win_ring == 0) return DSV4_ERR_SHAPE;
+  const void* ptrs[] = {q, kv_win, pool, idx, sink, qpos, q_index, out};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  return DSV4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsv4_status_string(dsv4_status s) {
+  switch (s) {
+    case DSV4_OK: return "ok";
+    case DSV4_ERR_ARG: return "invalid argument (null pointer or bad flag)";
+    case DSV4_ERR_SHAPE: return "unsupported or inconsistent sizes";
+    case DSV4_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case DSV4_ERR_DTYPE: return "unknown dtype";
+    case DSV4_ERR_CUDA: return "CUDA runtime error";
+    case DSV4_ERR_DEVICE_CHECK: return "device-side check failed";
+    case DSV4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t dsv4_version(void) { return 100; }
+
+uint64_t dsv4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t dsv4_workspace_bytes(const dsv4_params* p) {
+  if (!p || check_common(p) != DSV4_OK) return 0;
+  return align_up(layer_idx_bytes(p)) + align_up(scores_bytes(p));
+}
+
+dsv4_status dsv4_compress_kv(const dsv4_params* p, int32_t c, const void* x, const void* z, const float* bias,
+                             const int64_t* pos, int32_t apply_rope, void* pool, void* x_rot, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  return run_compress(p, c, x, z, bias, pos, apply_rope, pool, x_rot, stream);
+}
+
+dsv4_status dsv4_indexer_topk(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
+                              const int32_t* q_index, int32_t* idx, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if ((st = check_indexer(p)) != DSV4_OK) return st;
+  if (!qI || !wI || !poolI || !idx) return DSV4_ERR_ARG;
+  const void* ptrs[] = {qI, wI, poolI, q_index, idx, workspace};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (!q_index && p->Sq > p->S) return DSV4_ERR_SHAPE;
+  const size_t need = scores_bytes(p);
+  if (need > 0 && (!workspace || ws_bytes < need)) return DSV4_ERR_WORKSPACE;
+  return run_indexer(p, qI, wI, poolI, q_index, idx, workspace, ws_bytes, stream);
+}
+
+dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
+                                 const int32_t* idx, const float* sink, const int64_t* qpos,
+                                 const int32_t* q_index, void* out, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if ((st = check_attn(p)) != DSV4_OK) return st;
+  if ((st = check_attn_ptrs(p, q, kv_win, pool, idx, sink, qpos, q_index, out)) != DSV4_OK) return st;
+  return run_attn(p, q, kv_win, pool, idx, sink, qpos, q_index, out, stream);
+}
+
+dsv4_status dsv4_csa_layer(const dsv4_params* p, const void* q, const void* kv, const void* z, const float* bias,
+                           const void* qI, const float* wI, const void* kI, const void* zI, const float* biasI,
+                           const float* sink, const int64_t* pos, void* out, void* pool, void* poolI,
+                           void* kv_rot, int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if (p->Sq != p->S || p->win_ring != 0 || p->rope_q != 1) return DSV4_ERR_SHAPE;
+  if ((st = check_attn(p)) != DSV4_OK) return st;
+  if ((st = check_indexer(p)) != DSV4_OK) return st;
+  if (!q || !kv || !qI || !wI || !kI || !sink || !pos || !out || !pool || !poolI || !kv_rot) return DSV4_ERR_ARG;
+  const void* ptrs[] = {q, kv, z, bias, qI, wI, kI, zI, biasI, sink, pos, out, pool, poolI, kv_rot, idx, workspace};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
+  const size_t need = dsv4_workspace_bytes(p);
+  if (need > 0 && (!workspace || ws_bytes < need)) return DSV4_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx_buf = idx ? idx : reinterpret_cast<int32_t*>(ws);
+  char* scores = ws + align_up(layer_idx_bytes(p));
+  const size_t scores_cap = ws_bytes - align_up(layer_idx_bytes(p));
+
+  if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
+  if ((st = run_compress(p, p->cI, kI, zI, biasI, pos, 0, poolI, nullptr, stream)) != DSV4_OK) return st;
+  if ((st = run_indexer(p, qI, wI, poolI, nullptr, idx_buf, scores, scores_cap, stream)) != DSV4_OK) return st;
+  return run_attn(p, q, kv_rot, pool, idx_buf, sink, pos, nullptr, out, stream);
+}
+
+dsv4_status dsv4_hca_layer(const dsv4_params* p, const void* q, const void* kv, const void* z, const float* bias,
+                           const float* sink, const int64_t* pos, void* out, void* pool, void* kv_rot,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if (p->Sq != p->S || p->win_ring != 0 || p->rope_q != 1 || p->overlap != 0) return DSV4_ERR_SHAPE;
+  if ((st = check_attn(p)) != DSV4_OK) return st;
+  if (!q || !kv || !sink || !pos || !out || !pool || !kv_rot) return DSV4_ERR_ARG;
+  const void* ptrs[] = {q, kv, z, bias, sink, pos, out, pool, kv_rot};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
+  if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
+  return run_attn(p, q, kv_rot, pool, nullptr, sink, pos, nullptr, out, stream);
+}
+
+}  // extern "C"

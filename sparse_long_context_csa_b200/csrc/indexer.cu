@@ -1,0 +1,309 @@
+// Lightning Indexer scores and per-query top-k selection.
+//
+// Method: "DeepSeek-V4" doc, "Hybrid attention (§2.3)" CSA item — the Lightning Indexer
+// (eqs. 13-17) scores each query against the compressed pool and keeps the top
+// index_topk entries (eq. 17); "Attention mask layout" — -1 sentinels while fewer
+// entries are ready.  "DeepSeek-V3.2" doc, "DeepSeek Sparse Attention (DSA)" — a
+// low-head-count scorer with per-head weights; since the Hadamard rotation of the
+// reference indexer is orthogonal, the scores are computed directly.
+//
+// Score kernel (CUDA cores, fp32 accumulation): a CTA owns 128 pool entries (one per
+// thread) and 64 (query, head) rows.  The entry tile is staged once in shared memory,
+// each thread keeps its 64 dot products in registers, and the ReLU / head weights /
+// head sum happen in the epilogue, so the per-query score row is the only output.
+//
+// Top-k kernel: one CTA per query row.  Radix select over an order-preserving 32-bit
+// key of the fp32 score (4 passes of 8 bits) finds the K-th largest score T; every
+// entry above T is kept, and of the entries equal to T the lowest indices are kept
+// (the tie rule).  The kept entries are written in ascending entry order, which also
+// gives the attention gathers increasing addresses.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4 {
+
+namespace {
+
+constexpr int kTileW = 128;  // entries per score CTA
+constexpr int kRowsQH = 64;  // (query, head) rows per score CTA
+
+template <typename T, int NI, int CI>
+__global__ void __launch_bounds__(kTileW) indexer_scores_kernel(IndexerArgs a, int64_t row0, int64_t row1) {
+  constexpr int QB = kRowsQH / NI;  // queries per CTA
+  extern __shared__ float smem[];
+  float* qs = smem;                               // [64][CI]
+  float* ks = qs + kRowsQH * CI;                  // [128][CI+1]
+  __shared__ float ws[kRowsQH];
+  __shared__ int vis_s[QB];
+  __shared__ int maxvis_s;
+
+  const int tile = blockIdx.x;
+  const int64_t rbase = row0 + (int64_t)blockIdx.y * QB;
+  const int tid = threadIdx.x;
+
+  if (tid == 0) maxvis_s = 0;
+  __syncthreads();
+  if (tid < QB) {
+    const int64_t row = rbase + tid;
+    int v = 0;
+    if (row < row1) {
+      const int s = (int)(row % a.Sq);
+      const int t = query_cache_index(a.q_index, row, s);
+      v = visible_entries(t, a.m, a.P_cap);
+    }
+    vis_s[tid] = v;
+    atomicMax(&maxvis_s, v);
+  }
+  __syncthreads();
+  const int w0 = tile * kTileW;
+  if (w0 >= maxvis_s) return;  // nothing in this tile is visible to any query of the CTA
+
+  // stage query rows and head weights (rows past row1 are zero)
+  const T* qI = static_cast<const T*>(a.qI);
+  for (int i = tid; i < kRowsQH * CI; i += kTileW) {
+    const int r = i / CI;
+    const int64_t row = rbase + r / NI;
+    qs[i] = row < row1 ? to_f32<T>(qI[(rbase * NI) * CI + i]) : 0.f;
+  }
+  if (tid < kRowsQH) {
+    const int64_t row = rbase + tid / NI;
+    ws[tid] = row < row1 ? a.wI[rbase * NI + tid] : 0.f;
+  }
+  __syncthreads();
+
+  // The rows of a CTA may belong to several sequences (always when Sq < QB): the entry
+  // tile is staged and scored once per distinct sequence.  Entries past P_cap are zero.
+  const int64_t seq_first = rbase / a.Sq;
+  const int64_t last_row = (rbase + QB - 1 < row1 ? rbase + QB - 1 : row1 - 1);
+  const int64_t seq_last = last_row / a.Sq;
+  const T* poolI = static_cast<const T*>(a.poolI);
+  for (int64_t sq = seq_first; sq <= seq_last; ++sq) {
+    __syncthreads();
+    for (int i = tid; i < kTileW * CI; i += kTileW) {
+      const int e = i / CI, d = i % CI;
+      const int w = w0 + e;
+      ks[e * (CI + 1) + d] = w < a.P_cap ? to_f32<T>(poolI[((int64_t)sq * a.P_cap + w) * CI + d]) : 0.f;
+    }
+    __syncthreads();
+
+    float acc[kRowsQH];
+#pragma unroll
+    for (int i = 0; i < kRowsQH; ++i) acc[i] = 0.f;
+    const float* krow = ks + tid * (CI + 1);
+#pragma unroll 2
+    for (int d = 0; d < CI; d += 4) {
+      const float k0 = krow[d], k1 = krow[d + 1], k2 = krow[d + 2], k3 = krow[d + 3];
+#pragma unroll
+      for (int i = 0; i < kRowsQH; ++i) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + i * CI + d);
+        acc[i] = fmaf(k0, qv.x, acc[i]);
+        acc[i] = fmaf(k1, qv.y, acc[i]);
+        acc[i] = fmaf(k2, qv.z, acc[i]);
+        acc[i] = fmaf(k3, qv.w, acc[i]);
+      }
+    }
+    const int w = w0 + tid;
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      float sc = 0.f;
+#pragma unroll
+      for (int h = 0; h < NI; ++h) sc = fmaf(ws[q * NI + h], fmaxf(acc[q * NI + h], 0.f), sc);
+      const int64_t row = rbase + q;
+      if (row < row1 && row / a.Sq == sq && w < vis_s[q]) a.scores[(row - row0) * a.P_cap + w] = sc;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;  // -0 and +0 are the same score
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kTopkThreads = 512;
+constexpr int kTopkSmemKeys = 40960;  // keys cached in shared memory (160 KB)
+
+// Exclusive block scan of a 0/1 flag; returns the prefix and writes the block total.
+__device__ __forceinline__ int block_flag_scan(bool f, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, f);
+  const int in_warp = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[wid] = __popc(bal);
+  __syncthreads();
+  if (wid == 0) {
+    const int nw = kTopkThreads / 32;
+    int v = lane < nw ? warp_tot[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane < nw) warp_tot[lane] = incl - v;  // exclusive
+    if (lane == 31) *total = incl;
+  }
+  __syncthreads();
+  const int r = warp_tot[wid] + in_warp;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64_t row0) {
+  extern __shared__ uint32_t keys[];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need;
+  __shared__ int warp_tot[32];
+  __shared__ int s_total;
+
+  const int64_t row = row0 + blockIdx.x;
+  const int s = (int)(row % a.Sq);
+  const int t = query_cache_index(a.q_index, row, s);
+  const int vis = visible_entries(t, a.m, a.P_cap);
+  const int K = a.topk;
+  int32_t* out = a.idx + row * (int64_t)K;
+  const int tid = threadIdx.x;
+
+  if (vis <= K) {
+    for (int i = tid; i < K; i += kTopkThreads) out[i] = i < vis ? i : -1;
+    return;
+  }
+  const float* sc = a.scores + (int64_t)blockIdx.x * a.P_cap;
+  const bool cached = vis <= kTopkSmemKeys;
+  if (cached)
+    for (int i = tid; i < vis; i += kTopkThreads) keys[i] = order_key(sc[i]);
+  __syncthreads();
+
+  uint32_t prefix = 0u, mask = 0u;
+  int need = K;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < vis; i += kTopkThreads) {
+      const uint32_t k = cached ? keys[i] : order_key(sc[i]);
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns bins 255-8l-7 .. 255-8l (a descending run of 8)
+      const int top = 255 - 8 * tid;
+      int cnt[8];
+      int sum = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        cnt[k] = (int)hist[top - k];
+        sum += cnt[k];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += n;
+      }
+      const int excl = incl - sum;
+      if (excl < need && need <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (run < need && need <= run + cnt[k]) {
+            s_prefix = prefix | ((uint32_t)(top - k) << shift);
+            s_need = need - run;
+          }
+          run += cnt[k];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  // prefix = key of the K-th largest score; keep all keys > prefix and the `need`
+  // lowest-index keys == prefix, in ascending entry order.
+  int eq_seen = 0, taken = 0;
+  for (int base = 0; base < vis; base += kTopkThreads) {
+    const int i = base + tid;
+    uint32_t k = 0u;
+    if (i < vis) k = cached ? keys[i] : order_key(sc[i]);
+    const bool gt = i < vis && k > prefix;
+    const bool eq = i < vis && k == prefix;
+    const int eq_rank = eq_seen + block_flag_scan(eq, warp_tot, &s_total);
+    const int eq_tot = s_total;
+    const bool take = gt || (eq && eq_rank < need);
+    const int pos = taken + block_flag_scan(take, warp_tot, &s_total);
+    const int take_tot = s_total;
+    if (take && pos < K) out[pos] = i;
+    eq_seen += eq_tot;
+    taken += take_tot;
+    __syncthreads();
+  }
+}
+
+template <typename T, int NI, int CI>
+cudaError_t launch_scores_t(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  constexpr int QB = kRowsQH / NI;
+  const size_t smem = (size_t)(kRowsQH * CI + kTileW * (CI + 1)) * sizeof(float);
+  cudaFuncSetAttribute(indexer_scores_kernel<T, NI, CI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)smem);
+  dim3 grid((a.P_cap + kTileW - 1) / kTileW, (unsigned)((r1 - r0 + QB - 1) / QB));
+  indexer_scores_kernel<T, NI, CI><<<grid, kTileW, smem, st>>>(a, r0, r1);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <typename T, int CI>
+cudaError_t launch_scores_ci(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  switch (a.nI) {
+    case 1: return launch_scores_t<T, 1, CI>(a, r0, r1, st);
+    case 2: return launch_scores_t<T, 2, CI>(a, r0, r1, st);
+    case 4: return launch_scores_t<T, 4, CI>(a, r0, r1, st);
+    case 8: return launch_scores_t<T, 8, CI>(a, r0, r1, st);
+    case 16: return launch_scores_t<T, 16, CI>(a, r0, r1, st);
+    case 32: return launch_scores_t<T, 32, CI>(a, r0, r1, st);
+    case 64: return launch_scores_t<T, 64, CI>(a, r0, r1, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+template <typename T>
+cudaError_t launch_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  switch (a.cI) {
+    case 32: return launch_scores_ci<T, 32>(a, r0, r1, st);
+    case 64: return launch_scores_ci<T, 64>(a, r0, r1, st);
+    case 128: return launch_scores_ci<T, 128>(a, r0, r1, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace
+
+int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes) {
+  const int64_t per_row = (int64_t)P_cap * (int64_t)sizeof(float);
+  int64_t r = per_row > 0 ? (int64_t)(bytes / per_row) : total_rows;
+  if (r > total_rows) r = total_rows;
+  if (r > 65535) r = 65535;  // the score grid's y extent is rows / (64 / nI) <= 65535
+  return r;
+}
+
+cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st) {
+  const int64_t rows = (int64_t)a.B * a.Sq;
+  const size_t topk_smem = (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
+  cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)topk_smem);
+  for (int64_t r0 = 0; r0 < rows; r0 += a.rows_per_chunk) {
+    const int64_t r1 = r0 + a.rows_per_chunk < rows ? r0 + a.rows_per_chunk : rows;
+    cudaError_t e = dtype == DSV4_BF16 ? launch_scores<__nv_bfloat16>(a, r0, r1, st)
+                                       : launch_scores<float>(a, r0, r1, st);
+    if (e != cudaSuccess) return e;
+    topk_kernel<<<(unsigned)(r1 - r0), kTopkThreads, topk_smem, st>>>(a, r0);
+    note_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace dsv4

@@ -1,0 +1,59 @@
+// Launchers shared between the C-ABI layer (dsv4_api.cu) and the kernel files.
+// Arguments arrive validated; each launcher returns the cudaGetLastError() of its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dsv4.h"
+
+namespace dsv4 {
+
+// Count one kernel launch (read back by dsv4_launch_count).
+void note_launch(int n = 1);
+
+struct CompressArgs {
+  int B, S, c, m, overlap, P_cap, R, apply_rope;
+  float theta;
+  const void* x;
+  const void* z;
+  const float* bias;
+  const int64_t* pos;
+  void* pool;
+  void* x_rot;
+};
+cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st);
+
+struct IndexerArgs {
+  int B, Sq, nI, cI, m, P_cap, topk;
+  const void* qI;
+  const float* wI;
+  const void* poolI;
+  const int32_t* q_index;
+  int32_t* idx;
+  float* scores;        // workspace: [rows_per_chunk, P_cap] fp32
+  int64_t rows_per_chunk;
+};
+cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st);
+// Rows of queries whose scores fit in `bytes` of score workspace.
+int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes);
+
+struct AttnArgs {
+  int B, Sq, H, D, R, dv, n_win, win_ring, m, P_cap, topk, rope_q, rotate_out, kv_rows;
+  float scale, theta;
+  const void* q;
+  const void* kv_win;
+  const void* pool;
+  const int32_t* idx;
+  const float* sink;
+  const int64_t* qpos;
+  const int32_t* q_index;
+  void* out;
+};
+cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
+// Tensor-core (tcgen05) path; returns cudaErrorNotSupported when the shape is not covered.
+bool attn_tc_supported(const AttnArgs& a, int dtype);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
+
+}  // namespace dsv4

@@ -234,3 +234,39 @@ def make_inputs(w: Workload, gains: dict | None = None, threads: int = 8) -> dic
     if w.kind != "decode":
         out["pos"] = token_positions(w)
     return out
+
+
+def strided_selection(w: Workload, q_index: np.ndarray, stream: int = 15) -> np.ndarray:
+    """A valid index list per query for attention-only tests: [B,Sq,topk] int32.
+
+    Query (b,s) at cache index t keeps n = min(topk, vis) of its vis visible entries,
+    entry k = floor((k + u) * vis / n) for a seeded offset u in [0,1): distinct,
+    ascending, spread over the whole visible range; the remaining slots are -1.
+    """
+    rng = np.random.default_rng([w.seed, stream, 0])
+    t = q_index.reshape(-1).astype(np.int64)
+    vis = np.minimum((t + 1) // w.m, w.P_cap)
+    n = np.minimum(vis, w.topk)
+    u = rng.random(t.shape[0])
+    k = np.arange(w.topk, dtype=np.float64)[None, :]
+    nn = np.maximum(n, 1)[:, None].astype(np.float64)
+    sel = np.floor((k + u[:, None]) * vis[:, None] / nn).astype(np.int64)
+    sel = np.where(k < n[:, None], sel, -1)
+    return sel.reshape(w.B, w.Sq, w.topk).astype(np.int32)
+
+
+def cache_specs(w: Workload, gains: dict | None = None) -> dict:
+    """Specs of a pre-filled cache for kernel-level tests of any workload:
+    pool [B*P_cap, D], poolI [B*P_cap, cI] and window rows [B*(win_ring or S), D]."""
+    gains = gains or {}
+    bf = w.dtype == "bf16"
+
+    def spec(name, shape, scale):
+        return TensorSpec(w.seed, STREAMS[name], tuple(shape), float(scale) * gains.get(name, 1.0), bf)
+
+    rows = w.win_ring if w.win_ring else w.S
+    out = {"pool": spec("pool", (w.B * w.P_cap, w.D), 1 / math.sqrt(w.D)),
+           "win": spec("win", (w.B * rows, w.D), 1 / math.sqrt(w.D))}
+    if w.nI > 0:
+        out["poolI"] = spec("poolI", (w.B * w.P_cap, w.cI), 1 / math.sqrt(w.cI))
+    return out

@@ -1,0 +1,117 @@
+"""Host-side checks of libdsv4 that need no GPU: the library builds for sm_100a, loads,
+exports every entry point include/dsv4.h declares, and rejects bad calls on the host
+(those calls return before any CUDA call, so they are safe without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from sparse_long_context_csa_b200 import abi, build
+    build.build()
+    abi.load()
+    return abi
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsv4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsv4_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(abi):
+    names = _declared()
+    assert {"dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
+            "dsv4_hca_layer"} <= set(names)
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(abi.EXPORTED) == set(names)
+
+
+def test_version_and_status_strings(abi):
+    lib = abi.load()
+    assert lib.dsv4_version() >= 100
+    for code in range(8):
+        assert lib.dsv4_status_string(code)
+    assert b"unknown" in lib.dsv4_status_string(99)
+
+
+def _params(abi, **kw):
+    import synth
+    from sparse_long_context_csa_b200 import harness
+    return harness.params_for(synth.WORKLOADS["csa_prefill_bf16"], **kw)
+
+
+FAKE = 0x10000  # 16-byte aligned fake device address: never dereferenced, validation fails first
+
+
+def _attn(abi, p, **over):
+    a = dict(q=FAKE, kv_win=FAKE, pool=FAKE, idx=FAKE, sink=FAKE, qpos=FAKE, q_index=None, out=FAKE)
+    a.update(over)
+    lib = abi.load()
+    return lib.dsv4_sparse_mqa_attn(ctypes.byref(p) if p is not None else None, a["q"], a["kv_win"], a["pool"],
+                                    a["idx"], a["sink"], a["qpos"], a["q_index"], a["out"], None, 0, None)
+
+
+def test_attention_rejects_bad_arguments(abi):
+    assert _attn(abi, None) == 1
+    assert _attn(abi, _params(abi, dtype=7)) == 4
+    assert _attn(abi, _params(abi, dv=500)) == 2                 # dv not a multiple of 32
+    assert _attn(abi, _params(abi, dv=256)) == 2                 # rotate_out needs dv == D
+    assert _attn(abi, _params(abi, R=63)) == 2                   # odd rope width
+    assert _attn(abi, _params(abi, win_ring=64)) == 2            # ring shorter than the window
+    assert _attn(abi, _params(abi), q=FAKE + 8) == 3             # misaligned
+    assert _attn(abi, _params(abi), q=None) == 1
+    assert _attn(abi, _params(abi), qpos=None) == 1              # rope_q needs positions
+    assert _attn(abi, _params(abi, m=0)) == 2
+
+
+def test_indexer_rejects_bad_arguments(abi):
+    lib = abi.load()
+
+    def call(p, ws=FAKE, ws_bytes=1 << 40, **over):
+        a = dict(qI=FAKE, wI=FAKE, poolI=FAKE, q_index=None, idx=FAKE)
+        a.update(over)
+        return lib.dsv4_indexer_topk(ctypes.byref(p), a["qI"], a["wI"], a["poolI"], a["q_index"], a["idx"],
+                                     ws, ws_bytes, None)
+
+    assert call(_params(abi, nI=3)) == 2
+    assert call(_params(abi, cI=96)) == 2
+    assert call(_params(abi, topk=0)) == 2
+    assert call(_params(abi), ws=None, ws_bytes=0) == 7
+    assert call(_params(abi), ws_bytes=1024) == 7
+    assert call(_params(abi), idx=None) == 1
+    assert call(_params(abi), wI=FAKE + 4) == 3
+
+
+def test_compress_and_layers_reject_bad_arguments(abi):
+    lib = abi.load()
+    p = _params(abi)
+    assert lib.dsv4_compress_kv(ctypes.byref(p), 511, FAKE, None, None, FAKE, 1, FAKE, None, None) == 2
+    assert lib.dsv4_compress_kv(ctypes.byref(p), 512, FAKE, None, None, None, 1, FAKE, None, None) == 1
+    assert lib.dsv4_compress_kv(ctypes.byref(p), 512, FAKE, None, None, FAKE, 0, FAKE, FAKE, None) == 1
+    small = _params(abi, P_cap=100)  # S/m = 2048 entries do not fit
+    assert lib.dsv4_compress_kv(ctypes.byref(small), 512, FAKE, None, None, FAKE, 1, FAKE, None, None) == 2
+    args = [FAKE] * 17  # q .. idx, workspace
+    assert lib.dsv4_csa_layer(ctypes.byref(_params(abi, Sq=1)), *args, 1 << 40, None) == 2   # prefill only
+    assert lib.dsv4_csa_layer(ctypes.byref(p), *args, 16, None) == 7                          # workspace too small
+    assert lib.dsv4_csa_layer(ctypes.byref(p), *args[:16], None, 1 << 40, None) == 7
+    assert lib.dsv4_hca_layer(ctypes.byref(p), *([FAKE] * 10), 0, None) == 2              # overlap=1 is CSA
+
+
+def test_workspace_is_a_pure_function_of_params(abi):
+    import synth
+    from sparse_long_context_csa_b200 import harness
+    sizes = {n: abi.dsv4_workspace_bytes(harness.params_for(w)) for n, w in synth.WORKLOADS.items()}
+    assert sizes["hca_prefill_bf16"] == 0                      # no indexer
+    assert sizes["csa_prefill_bf16"] == 8192 * 512 * 4 + 8192 * 2048 * 4
+    assert sizes["csa_decode_bf16"] == 64 * 32768 * 4           # decode keeps no layer idx
+    assert sizes["dsa_prefill_bf16"] == 32768 * 2048 * 4 + (256 << 20)
+    assert abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"])) == \
+        abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"]))
