@@ -27,6 +27,13 @@ pytestmark = pytest.mark.gpu
 ATTN_TOL = {"f32": 1e-5, "bf16": 2e-3}
 STORE_RTOL = {"f32": 2.0 ** -23, "bf16": 2.0 ** -7}
 STORE = {"f32": "f32", "bf16": "bf16"}
+U32 = 2.0 ** -24
+
+
+def fp32_atol(x, n_terms):
+    """Absolute error bound of an fp32 sum of n_terms products of inputs |x| (weights <= 1),
+    which the relative storage tolerance does not cover when the result cancels to ~0."""
+    return (n_terms + 8) * U32 * float(np.abs(np.asarray(x)).max())
 
 
 @pytest.fixture(scope="module")
@@ -88,9 +95,10 @@ def test_tiny_csa_layer_f32(lib, gains):
                       host["zI"], host["biasI"], host["sink"], host["pos"], overlap=w.overlap, topk=w.topk,
                       store="f32", **_oracle_kw(w))
     P = w.S // w.m
-    assert_close_rel(_np(o["pool"])[:, :P], ref["pool"], STORE_RTOL["f32"] * 4, 1e-7, "pool")
-    assert_close_rel(_np(o["poolI"])[:, :P], ref["poolI"], STORE_RTOL["f32"] * 4, 1e-7, "poolI")
-    assert_close_rel(_np(o["kv_rot"]), ref["kv_rot"], STORE_RTOL["f32"] * 4, 1e-7, "kv_rot")
+    nt = 2 * w.m if w.overlap else w.m
+    assert_close_rel(_np(o["pool"])[:, :P], ref["pool"], STORE_RTOL["f32"], fp32_atol(host["kv"], nt), "pool")
+    assert_close_rel(_np(o["poolI"])[:, :P], ref["poolI"], STORE_RTOL["f32"], fp32_atol(host["kI"], nt), "poolI")
+    assert_close_rel(_np(o["kv_rot"]), ref["kv_rot"], STORE_RTOL["f32"], fp32_atol(host["kv"], 2), "kv_rot")
     rows = [(0, s) for s in range(w.S)]
     _check_layer_idx_and_out(w, host, o, ref, rows, rel_key_err=4 * 2.0 ** -24)
 
@@ -103,9 +111,10 @@ def test_csa_prefill_layer_bf16(lib):
                       host["zI"], host["biasI"], host["sink"], host["pos"], overlap=w.overlap, topk=w.topk,
                       store="bf16", rows=rows, **_oracle_kw(w))
     P = w.S // w.m
-    assert_close_rel(_np(o["pool"])[:, :P], ref["pool"], STORE_RTOL["bf16"], 1e-30, "pool")
-    assert_close_rel(_np(o["poolI"])[:, :P], ref["poolI"], STORE_RTOL["bf16"], 1e-30, "poolI")
-    assert_close_rel(_np(o["kv_rot"]), ref["kv_rot"], STORE_RTOL["bf16"], 1e-30, "kv_rot")
+    nt = 2 * w.m if w.overlap else w.m
+    assert_close_rel(_np(o["pool"])[:, :P], ref["pool"], STORE_RTOL["bf16"], fp32_atol(host["kv"], nt), "pool")
+    assert_close_rel(_np(o["poolI"])[:, :P], ref["poolI"], STORE_RTOL["bf16"], fp32_atol(host["kI"], nt), "poolI")
+    assert_close_rel(_np(o["kv_rot"]), ref["kv_rot"], STORE_RTOL["bf16"], fp32_atol(host["kv"], 2), "kv_rot")
     _check_layer_idx_and_out(w, host, o, ref, rows, rel_key_err=STORE_RTOL["bf16"])
 
 
@@ -115,9 +124,9 @@ def test_hca_prefill_layer_bf16(lib):
     rows = [(0, s) for s in sample_rows(w.S, 256, 64)]
     ref = O.hca_layer(host["q"], host["kv"], host["z"], host["bias"], host["sink"], host["pos"], rows=rows,
                       store="bf16", **_oracle_kw(w))
-    assert_close_rel(_np(o["pool"]), ref["pool"], STORE_RTOL["bf16"], 1e-30, "pool")
+    assert_close_rel(_np(o["pool"]), ref["pool"], STORE_RTOL["bf16"], fp32_atol(host["kv"], w.m), "pool")
     gkv = _np(o["kv_rot"])
-    assert_close_rel(gkv[:, ::97], ref["kv_rot"][:, ::97], STORE_RTOL["bf16"], 1e-30, "kv_rot")
+    assert_close_rel(gkv[:, ::97], ref["kv_rot"][:, ::97], STORE_RTOL["bf16"], fp32_atol(host["kv"], 2), "kv_rot")
     gout = _np(o["out"])
     for b, s in rows:
         assert_max_abs(gout[b, s], ref["out"][b, s], ATTN_TOL["bf16"], f"out row {s}")
@@ -130,7 +139,7 @@ def test_dsa_prefill_layer_bf16(lib):
     ref = O.csa_layer(host["q"], host["kv"], None, None, host["qI"], host["wI"], host["kI"], None, None,
                       host["sink"], host["pos"], overlap=0, topk=w.topk, store="bf16", rows=rows,
                       **_oracle_kw(w))
-    assert_close_rel(_np(o["pool"]), ref["pool"], STORE_RTOL["bf16"], 1e-30, "pool")
+    assert_close_rel(_np(o["pool"]), ref["pool"], STORE_RTOL["bf16"], fp32_atol(host["kv"], 2), "pool")
     # m = 1: the indexer pool is the key stream itself
     np.testing.assert_array_equal(_np(o["poolI"]), host["kI"])
     _check_layer_idx_and_out(w, host, o, ref, rows, rel_key_err=STORE_RTOL["bf16"])
@@ -224,11 +233,12 @@ def test_compress_kernel_ragged(lib, dtype, overlap, m):
     P = w.S // m
     ref = O.compress(host["kv"], host.get("z"), host.get("bias"), host["pos"], m=m, overlap=overlap,
                      apply_rope=True, R=w.R, theta=w.theta)
-    tol = STORE_RTOL[dtype] * (4 if dtype == "f32" else 1)
-    assert_close_rel(_np(pool)[:, :P], ref, tol, 1e-7 if dtype == "f32" else 1e-30, "pool")
+    tol = STORE_RTOL[dtype]
+    nt = 2 * m if overlap else m
+    assert_close_rel(_np(pool)[:, :P], ref, tol, fp32_atol(host["kv"], nt), "pool")
     assert np.all(_np(pool)[:, P:] == 0), "entries past S/m must be left untouched"
     assert_close_rel(_np(xr), O.rope_rotate(host["kv"], host["pos"], w.R, w.theta), tol,
-                     1e-7 if dtype == "f32" else 1e-30, "x_rot")
+                     fp32_atol(host["kv"], 2), "x_rot")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
