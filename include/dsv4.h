@@ -123,6 +123,27 @@ dsv4_status dsv4_indexer_topk(const dsv4_params* params, const void* qI, const f
                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Allocation-free variant of dsv4_indexer_topk (the method has no counterpart: this is a
+ * deployment convenience).  It is for callers that cannot hand the library a workspace:
+ * plugin hosts that own all device memory and expose no allocator to the kernels they
+ * call, and decode loops that must not call cudaMalloc / cudaFree because those calls can
+ * synchronise the whole device.  Same arguments, results and ordering as
+ * dsv4_indexer_topk, minus the workspace: the fp32 score rows live in a fixed 16 MiB
+ * array of device memory inside the library (4,194,304 scores; every GPU that loads the
+ * library holds it until the process exits), processed in chunks of whole query rows.
+ *   - P_cap above 4,194,304 is rejected with DSV4_ERR_SHAPE (one score row must fit).
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call before any
+ *     stream capture.  It allocates nothing, then or later.
+ *   - Every call shares the array.  Calls that overlap on the GPU (other streams, other
+ *     host threads) race on it and must be serialised by the caller.  No part of the
+ *     array needs to start at zero: each score row is written before it is read.
+ */
+dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* params, const void* qI, const float* wI,
+                                      const void* poolI, const int32_t* q_index, int32_t* idx,
+                                      void* stream);
+
+/*
  * Sparse shared-K=V MQA attention with sink ([V4] "Hybrid attention (§2.3)": one KV
  * head read as key and value, partial RoPE, -i output rotation (eq. 26), per-head sink
  * (eq. 27), sliding-window K=V branch concatenated with the compressor entries).

@@ -20,7 +20,7 @@ STATUS = {0: "DSV4_OK", 1: "DSV4_ERR_ARG", 2: "DSV4_ERR_SHAPE", 3: "DSV4_ERR_ALI
 
 EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
-            "dsv4_launch_count")
+            "dsv4_launch_count", "dsv4_indexer_topk_noalloc")
 
 
 class Dsv4Error(RuntimeError):
@@ -56,6 +56,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     lib.dsv4_compress_kv.argtypes = [P, i32, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.dsv4_indexer_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsv4_indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.dsv4_sparse_mqa_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_csa_layer.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.dsv4_hca_layer.argtypes = [P] + [vp] * 10 + [sz, vp]
@@ -66,7 +67,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_version.restype = i32
     lib.dsv4_launch_count.restype = ctypes.c_uint64
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
-               "dsv4_hca_layer"):
+               "dsv4_hca_layer", "dsv4_indexer_topk_noalloc"):
         getattr(lib, fn).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -112,6 +113,12 @@ def dsv4_indexer_topk(params, qI, wI, poolI, q_index, idx, workspace, ws_bytes=N
     _check("dsv4_indexer_topk", load().dsv4_indexer_topk(
         ctypes.byref(params), _ptr(qI), _ptr(wI), _ptr(poolI), _ptr(q_index), _ptr(idx), _ptr(workspace),
         ws_bytes, _stream(stream)))
+
+
+def dsv4_indexer_topk_noalloc(params, qI, wI, poolI, q_index, idx, stream=None):
+    """dsv4_indexer_topk without a workspace: scores go to the library's fixed device scratch."""
+    _check("dsv4_indexer_topk_noalloc", load().dsv4_indexer_topk_noalloc(
+        ctypes.byref(params), _ptr(qI), _ptr(wI), _ptr(poolI), _ptr(q_index), _ptr(idx), _stream(stream)))
 
 
 def dsv4_sparse_mqa_attn(params, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace=None,

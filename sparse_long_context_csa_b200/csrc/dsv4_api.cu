@@ -191,6 +191,23 @@ dsv4_status dsv4_indexer_topk(const dsv4_params* p, const void* qI, const float*
   return run_indexer(p, qI, wI, poolI, q_index, idx, workspace, ws_bytes, stream);
 }
 
+dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
+                                      const int32_t* q_index, int32_t* idx, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if ((st = check_indexer(p)) != DSV4_OK) return st;
+  if (!qI || !wI || !poolI || !idx) return DSV4_ERR_ARG;
+  const void* ptrs[] = {qI, wI, poolI, q_index, idx};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (!q_index && p->Sq > p->S) return DSV4_ERR_SHAPE;
+  if ((int64_t)p->P_cap > kNoAllocScoreFloats) return DSV4_ERR_SHAPE;  // one score row must fit
+  if ((int64_t)p->B * p->Sq == 0) return DSV4_OK;
+  float* scratch = nullptr;
+  if (noalloc_scores_scratch(&scratch) != cudaSuccess) return DSV4_ERR_CUDA;
+  return run_indexer(p, qI, wI, poolI, q_index, idx, scratch, (size_t)kNoAllocScoreFloats * sizeof(float), stream);
+}
+
 dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
                                  const int32_t* idx, const float* sink, const int64_t* qpos,
                                  const int32_t* q_index, void* out, void* workspace, size_t ws_bytes,

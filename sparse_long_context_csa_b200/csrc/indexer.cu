@@ -19,6 +19,8 @@
 // gives the attention gathers increasing addresses.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -280,6 +282,32 @@ cudaError_t launch_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStre
 }
 
 }  // namespace
+
+// Fixed score scratch of dsv4_indexer_topk_noalloc: a file-scope device array, so that
+// callers without an allocator still get the indexer.  Every device that loads the
+// library holds these bytes until the process exits.  Calls share the array; nothing in
+// it has to start at zero (each score row is written before it is read).
+static __device__ __align__(256) float g_noalloc_scores[kNoAllocScoreFloats];
+
+cudaError_t noalloc_scores_scratch(float** ptr) {
+  static std::mutex mu;
+  static float* by_device[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!by_device[dev]) {
+    // Host code sees g_noalloc_scores only as a stand-in symbol; the device address of this
+    // device's copy comes from the runtime, with this device current.
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scores);
+    if (e != cudaSuccess) return e;
+    by_device[dev] = static_cast<float*>(p);
+  }
+  *ptr = by_device[dev];
+  return cudaSuccess;
+}
 
 int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes) {
   const int64_t per_row = (int64_t)P_cap * (int64_t)sizeof(float);

@@ -38,6 +38,10 @@ struct IndexerArgs {
 cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st);
 // Rows of queries whose scores fit in `bytes` of score workspace.
 int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes);
+// Device address (on the current device) of the fixed score scratch used by
+// dsv4_indexer_topk_noalloc; set up on the first call per device.
+constexpr int64_t kNoAllocScoreFloats = int64_t(4) << 20;  // 16 MiB of fp32 scores
+cudaError_t noalloc_scores_scratch(float** ptr);
 
 struct AttnArgs {
   int B, Sq, H, D, R, dv, n_win, win_ring, m, P_cap, topk, rope_q, rotate_out, kv_rows;
