@@ -228,6 +228,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="for profilers: only the warm-up and timed steps (no clock sampler, e2e or cpu_baseline)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -269,12 +271,13 @@ def main():
 
     # warm-up (also starts the clock sampler and lets it settle)
     sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
-    sampler.start()
+    if not args.profile_run:
+        sampler.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     t_w = time.time()
-    while time.time() - t_w < 1.0:  # keep the GPU busy while nvidia-smi starts sampling
+    while not args.profile_run and time.time() - t_w < 1.0:  # keep the GPU busy while nvidia-smi starts
         step()
         torch.cuda.synchronize()
 
@@ -296,6 +299,10 @@ def main():
     ms = max_over_ranks(start.elapsed_time(end))
     attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
     clocks = sampler.summary(wall0, wall1)
+    if args.profile_run:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": ms / args.steps, "attn_ms": attn_ms}), flush=True)
+        return
 
     # end to end through the layer entry point: pinned host inputs in, output back
     host_t = harness.to_device(w, host, device=None, pin=True)

@@ -48,7 +48,7 @@ typedef enum {
   DSV4_ERR_ALIGN = 3,        /* a tensor pointer is not 16-byte aligned */
   DSV4_ERR_DTYPE = 4,        /* unknown params->dtype */
   DSV4_ERR_CUDA = 5,         /* the CUDA runtime refused a launch or query */
-  DSV4_ERR_DEVICE_CHECK = 6, /* reserved: a device-side check word reported a bad index */
+  DSV4_ERR_DEVICE_CHECK = 6, /* dsv4_device_check: a kernel gave up a bounded wait */
   DSV4_ERR_WORKSPACE = 7     /* workspace missing or smaller than dsv4_workspace_bytes() */
 } dsv4_status;
 
@@ -203,6 +203,11 @@ const char* dsv4_status_string(dsv4_status status);
 
 /* Library ABI version (major * 100 + minor). */
 int32_t dsv4_version(void);
+
+/* Synchronise `stream`, then read and clear the device-side check word of the current
+ * device: DSV4_ERR_DEVICE_CHECK means a kernel gave up a bounded pipeline wait (its CTA
+ * returned early and its outputs are invalid); nothing traps or hangs instead. */
+dsv4_status dsv4_device_check(void* stream);
 
 /* Kernels this process has enqueued through libdsv4 so far (all devices, all entry
  * points); a monotone counter for launch accounting, read without synchronising. */

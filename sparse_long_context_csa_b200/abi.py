@@ -20,7 +20,7 @@ STATUS = {0: "DSV4_OK", 1: "DSV4_ERR_ARG", 2: "DSV4_ERR_SHAPE", 3: "DSV4_ERR_ALI
 
 EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
-            "dsv4_launch_count", "dsv4_indexer_topk_noalloc")
+            "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check")
 
 
 class Dsv4Error(RuntimeError):
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_status_string.restype = ctypes.c_char_p
     lib.dsv4_version.restype = i32
     lib.dsv4_launch_count.restype = ctypes.c_uint64
+    lib.dsv4_device_check.argtypes = [vp]
+    lib.dsv4_device_check.restype = ctypes.c_int
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
                "dsv4_hca_layer", "dsv4_indexer_topk_noalloc"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -91,6 +93,11 @@ def _stream(stream) -> int | None:
 def _check(fn: str, st: int) -> None:
     if st != 0:
         raise Dsv4Error(fn, st, load().dsv4_status_string(st).decode())
+
+
+def dsv4_device_check(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel reported a device-side failure."""
+    _check("dsv4_device_check", load().dsv4_device_check(_stream(stream)))
 
 
 def dsv4_launch_count() -> int:

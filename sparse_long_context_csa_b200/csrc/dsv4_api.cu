@@ -163,6 +163,13 @@ int32_t dsv4_version(void) { return 100; }
 
 uint64_t dsv4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+dsv4_status dsv4_device_check(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return DSV4_ERR_CUDA;
+  int code = 0;
+  if (take_attn_tc_error(&code) != cudaSuccess) return DSV4_ERR_CUDA;
+  return code ? DSV4_ERR_DEVICE_CHECK : DSV4_OK;
+}
+
 size_t dsv4_workspace_bytes(const dsv4_params* p) {
   if (!p || check_common(p) != DSV4_OK) return 0;
   return align_up(layer_idx_bytes(p)) + align_up(scores_bytes(p));

@@ -59,5 +59,7 @@ cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 // Tensor-core (tcgen05) path; returns cudaErrorNotSupported when the shape is not covered.
 bool attn_tc_supported(const AttnArgs& a, int dtype);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
+// Read and clear the tensor-core kernel's error word (non-zero: a bounded wait gave up).
+cudaError_t take_attn_tc_error(int* code);
 
 }  // namespace dsv4

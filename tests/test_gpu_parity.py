@@ -56,7 +56,7 @@ def _run_layer(lib, w, gains=None):
     x = harness.to_device(w, host)
     o = harness.make_outputs(w, params)
     harness.step(w, params, x, o)
-    torch.cuda.synchronize()
+    abi.dsv4_device_check()
     return host, o
 
 
@@ -204,7 +204,7 @@ def test_sparse_attention_kernel(lib, name, gains, use_idx):
     didx = torch.from_numpy(idx).cuda() if use_idx else None
     out = torch.empty((w.B, w.Sq, w.H, w.dv), dtype=harness.torch_dtype(w), device="cuda")
     abi.dsv4_sparse_mqa_attn(params, d["q"], d["win"], d["pool"], didx, d["sink"], d["qpos"], d["q_index"], out)
-    torch.cuda.synchronize()
+    abi.dsv4_device_check()
     rows = [(b, s) for b in range(w.B) for s in (sample_rows(w.Sq, 192, 32) if w.Sq > 1 else [0])]
     ref = O.sparse_mqa_attention(x["q"], c["win"], c["pool"], idx, x["sink"], x["qpos"], x["q_index"],
                                  n_win=w.n_win, m=w.m, scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rope_q=True,
