@@ -7,23 +7,29 @@
 // entries picked by the Lightning Indexer; "DeepSeek-V3.2" doc, DSA item 2 (attention over
 // the selected tokens only).
 //
-// Design (one CTA per query token; its 64 heads share every key row):
-//  * The key set of a query (window rows, then the selected pool entries) is cut into
-//    tiles of 128 keys.  One producer warp gathers a tile's rows with TMA tile::gather4
-//    (4 arbitrary rows per instruction, 128-byte swizzle) straight into the operand layout.
-//  * Scores are computed transposed, S^T[key, head] = K_tile . Q^T, as one 128x64xD MMA
-//    chain (M = 128 keys keeps the tensor core at full rate; 64 heads alone would be an
-//    M=64 half-rate shape).  The same shared-memory tile is then read as V^T (MN-major)
-//    for O^T[dim, head] += V^T . P^T: K=V costs one gather for both products.
-//  * The softmax warps own one key (TMEM lane) each and hold its 64 head scores.  The
-//    running max per head starts at the sink logit and is only raised when some score
-//    exceeds it by more than 2^8 (then the O^T columns are rescaled in TMEM), so the common
-//    tile needs no cross-thread reduction.  Per-thread partial denominators are reduced
-//    once, in the epilogue, where the sink term e^{sink - max} is added.
-//  * Accumulators: S^T 64 TMEM columns, O^T dv/128 tiles x 64 columns.
-//  * The output leaves TMEM transposed; it is staged through shared memory and written
-//    with 16-byte coalesced stores, after the -qpos rotation of the rope slice.
-// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), 2-5 = softmax/epilogue.
+// Design.  A persistent CTA per SM walks its queries; the 64 heads of a query share every
+// key row (MQA).
+//  * Keys of a query = window rows, then the selected pool entries, cut into 128-key tiles.
+//    A producer warp gathers each tile with TMA tile::gather4 (4 arbitrary rows per
+//    instruction) in 64-channel chunks, straight into the 128B-swizzled operand layout.
+//    Every chunk has its own full/free barrier pair, so S^T starts on the first chunk that
+//    lands and the next tile's gathers refill a chunk as soon as PV has read it.
+//  * Scores are computed transposed, S^T[key, head] = K_tile . Q^T (M = 128 keys keeps the
+//    tensor core at full rate; 64 heads alone would be a half-rate M=64 shape), and the same
+//    shared-memory tile is read again as V^T (MN-major) for O^T[dim, head] += V^T . P^T: K=V
+//    costs one gather for both products.
+//  * q (64 heads x D) arrives by TMA in the same swizzled layout as soon as the previous
+//    query's last S^T has read the buffer; two prep warps rotate its rope slice in place and
+//    scan the query's index row while the previous query finishes.
+//  * Softmax warps own one key (TMEM lane) each.  The running max per head starts at the
+//    sink logit and is raised only when a score exceeds it by more than 2^8 (the O^T columns
+//    are then rescaled in TMEM), so a typical tile needs no cross-thread reduction.
+//  * TMEM: S^T 64 columns, O^T dv/128 tiles x 64 columns.  The epilogue reads O^T, applies
+//    1/denominator and the -qpos rotation, and stores straight to global memory.
+// Warp roles: 0 producer (TMA), 1 MMA issuer + TMEM owner, 2-5 softmax/epilogue,
+//             6-7 query prep (descriptor, RoPE of q).
+// Every wait is bounded; a role that gives up records g_attn_tc_error and all roles leave
+// their loops together (warp votes / barrier reductions), free TMEM and return.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -34,20 +40,25 @@
 
 namespace dsv4 {
 
-__device__ int g_attn_tc_error = 0;  // non-zero: a pipeline wait gave up (the CTA returned early)
+__device__ int g_attn_tc_error = 0;  // non-zero: a pipeline wait gave up (the CTA stopped early)
 
 namespace {
 
 constexpr int kH = 64;
 constexpr int kTile = 128;
-constexpr int kThreads = 192;
-constexpr int kSoftmaxWarp0 = 2;
+constexpr int kThreads = 256;
+constexpr int kMaxChunks = 9;  // D <= 576
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 20;
+
+struct TcParams {
+  AttnArgs a;
+  double inv_freq[64];  // theta^(-2k/R), k < R/2
+  int64_t nrows;        // B * Sq queries
+};
 
 struct Smem {
-  // byte offsets inside the dynamic shared memory window
   uint32_t q, k, p, misc, total;
 };
 
@@ -63,32 +74,41 @@ __host__ __device__ inline Smem smem_layout(int D) {
   return s;
 }
 
+struct QDesc {
+  int64_t qrow;
+  int t, vis, wlo, nw, nw4, npool, ntiles;
+  float cs[64], sn[64];  // RoPE table at the query position
+};
+
 struct Misc {
-  uint64_t kfull, sfull, pfull, odone;
+  uint64_t cfull[kMaxChunks], cfree[kMaxChunks];
+  uint64_t qfull, qready, qfree, sfull, pfull, odone;
+  uint64_t dfull[2], dfree[2];
   uint32_t tmem_base;
-  int npool_last;   // highest valid pool slot + 1
-  int abort_flag;
   int rescale_cnt[2];
-  uint32_t mask[4];     // validity of the 128 keys of the current tile
-  float m[kH];          // running max per head (log2 units)
-  float cs[64], sn[64]; // RoPE table of the query position
-  float inv_l[kH];
-  float fac[kH];        // rescale factor per head (rare path)
+  int npool_tmp;
+  float m[kH];
+  float fac[kH];
   float red[4][kH];
+  float inv_l[kH];
+  QDesc desc[2];
 };
 static_assert(sizeof(Misc) <= 4096, "misc block exceeds its reservation");
 
-__device__ __forceinline__ void set_error(Misc* ms, int code) {
-  atomicExch(&g_attn_tc_error, code);
-  ms->abort_flag = 1;
+__device__ __forceinline__ bool wait_ok(uint64_t* bar, uint32_t parity) {
+  return tc::mbar_wait(bar, parity, kWaitLimit);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_win, const __grid_constant__ CUtensorMap map_pool,
-                   const AttnArgs a) {
+                   const __grid_constant__ CUtensorMap map_q, const __grid_constant__ TcParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  const AttnArgs& a = P.a;
   const int D = a.D;
   const int nch = D / 64;
+  const bool alias = D > 512;
+  const int nvch = a.dv / 64;  // chunks that are also value channels
+  const int nvt = a.dv / 128;
   const Smem L = smem_layout(D);
   Misc* ms = reinterpret_cast<Misc*>(smem + L.misc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -97,27 +117,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) atomicExch(&g_attn_tc_error, 3);
     return;
   }
+  const int64_t nq_cta = P.nrows > (int64_t)blockIdx.x ? (P.nrows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-  const int64_t qrow = blockIdx.x;
-  const int b = (int)(qrow / a.Sq);
-  const int s = (int)(qrow % a.Sq);
-  const int t = query_cache_index(a.q_index, qrow, s);
-  const int vis = visible_entries(t, a.m, a.P_cap);
-  const int wlo = t - a.n_win + 1 > 0 ? t - a.n_win + 1 : 0;
-  const int win_rows = a.win_ring ? a.win_ring : a.kv_rows;
-  int nw = a.n_win > 0 ? t - wlo + 1 : 0;
-  if (nw < 0) nw = 0;
-  if (!a.win_ring && wlo + nw > a.kv_rows) nw = a.kv_rows > wlo ? a.kv_rows - wlo : 0;
-  const int nw4 = (nw + 3) & ~3;
-
-  // ---------------------------------------------------------------- prologue
   if (tid == 0) {
-    tc::mbar_init(&ms->kfull, 1);
+    for (int c = 0; c < kMaxChunks; ++c) {
+      tc::mbar_init(&ms->cfull[c], 1);
+      tc::mbar_init(&ms->cfree[c], 1);
+    }
+    tc::mbar_init(&ms->qfull, 1);
+    tc::mbar_init(&ms->qready, 64);
+    tc::mbar_init(&ms->qfree, 1);
     tc::mbar_init(&ms->sfull, 1);
     tc::mbar_init(&ms->pfull, 128);
     tc::mbar_init(&ms->odone, 1);
-    ms->npool_last = a.idx ? 0 : (vis > 0 ? vis : 0);
-    ms->abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&ms->dfull[i], 64);
+      tc::mbar_init(&ms->dfree[i], 3);
+    }
     ms->rescale_cnt[0] = ms->rescale_cnt[1] = 0;
     tc::mbar_fence_init();
   }
@@ -128,292 +144,398 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tc::prefetch_tensormap(&map_win);
     tc::prefetch_tensormap(&map_pool);
+    tc::prefetch_tensormap(&map_q);
   }
-  // RoPE table of the query position
-  const int R = a.R;
-  if (a.rope_q || a.rotate_out) {
-    for (int k = tid; k < R / 2; k += kThreads) {
-      float c, sn;
-      rope_cos_sin(a.qpos[qrow], k, R, a.theta, &c, &sn);
-      ms->cs[k] = c;
-      ms->sn[k] = sn;
-    }
-  }
-  for (int h = tid; h < kH; h += kThreads) ms->m[h] = a.sink[h] * kLog2e;
-  __syncthreads();
-  // last valid pool slot (slots past it are not processed; holes inside are masked)
-  if (a.idx) {
-    int last = 0;
-    const int32_t* ir = a.idx + qrow * a.topk;
-    for (int k = tid; k < a.topk; k += kThreads) {
-      const int w = ir[k];
-      if (w >= 0 && w < vis) last = k + 1;
-    }
-    if (last) atomicMax(&ms->npool_last, last);
-  }
-  // q rows (64 heads x D), rotated at qpos, into the 128B-swizzled K-major B-operand layout
-  {
-    const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + qrow * kH * D);
-    const int per_head = D / 8;
-    const int rope_lo = D - R;
-    for (int ci = tid; ci < kH * per_head; ci += kThreads) {
-      const int h = ci / per_head;
-      const int d0 = (ci % per_head) * 8;
-      uint4 v = qg[ci];
-      if (a.rope_q && d0 >= rope_lo) {
-        __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(p2[e]);
-          const int k = (d0 - rope_lo) / 2 + e;
-          const float c = ms->cs[k], sn = ms->sn[k];
-          p2[e] = __floats2bfloat162_rn(f.x * c - f.y * sn, f.x * sn + f.y * c);
-        }
-      }
-      const int ch = d0 / 64, u = (d0 % 64) / 8;
-      *reinterpret_cast<uint4*>(smem + L.q + ch * 8192 + h * 128 + ((u ^ (h & 7)) * 16)) = v;
-    }
-  }
-  tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-
-  const int npool = ms->npool_last;
-  const int NK = nw4 + npool;
-  const int ntiles = (NK + kTile - 1) / kTile;
   const uint32_t tmem = ms->tmem_base;
   const uint32_t tS = tmem, tO = tmem + 64;
-  const int nvt = a.dv / 128;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
-    const int win_base = b * win_rows;
-    const int pool_base = b * a.P_cap;
-    for (int i = 0; i < ntiles; ++i) {
-      // every lane takes the same decision, so no lane is left waiting in __syncwarp
-      if (!__all_sync(0xffffffffu, i == 0 || tc::mbar_wait(&ms->odone, (i - 1) & 1, kWaitLimit))) {
-        if (lane == 0) set_error(ms, 1);
+  if (warp >= 6) {
+    // ================================================================ query prep (64 threads)
+    const int pt = tid - 192;
+    const int R = a.R;
+    const int rope_lo = D - R;
+    bool ok = true;
+    for (int64_t n = 0; n < nq_cta; ++n) {
+      const int slot = (int)(n & 1);
+      const int64_t qrow = blockIdx.x + n * gridDim.x;
+      if (n >= 2 && !tc::named_bar_and(2, 64, wait_ok(&ms->dfree[slot], ((n >> 1) - 1) & 1))) {
+        ok = false;
         break;
       }
-      const int k0 = i * kTile;
-      const int nvalid = min(kTile, NK - k0);
-      const int nk = (nvalid + 15) & ~15;
-      // validity mask of the tile (lane l covers keys 4l..4l+3)
-      uint32_t bits = 0;
-      int rows[4];
-      const bool pool_grp = (k0 + 4 * lane) >= nw4 && npool > 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = k0 + 4 * lane + e;
-        bool valid = false;
-        int row;
-        if (pool_grp) {
-          const int p = k - nw4;
-          int w = 0;
-          if (k < NK) {
-            w = ir ? ir[p] : p;
-            valid = w >= 0 && w < vis;
-          }
-          row = pool_base + (valid ? w : 0);
-        } else {
-          valid = k < nw;
-          const int j = valid ? wlo + (k) : wlo;
-          row = win_base + (a.win_ring ? j % a.win_ring : j);
+      QDesc* d = &ms->desc[slot];
+      const int s = (int)(qrow % a.Sq);
+      const int t = query_cache_index(a.q_index, qrow, s);
+      const int vis = visible_entries(t, a.m, a.P_cap);
+      const int wlo = t - a.n_win + 1 > 0 ? t - a.n_win + 1 : 0;
+      int nw = a.n_win > 0 ? t - wlo + 1 : 0;
+      if (nw < 0) nw = 0;
+      if (!a.win_ring && wlo + nw > a.kv_rows) nw = a.kv_rows > wlo ? a.kv_rows - wlo : 0;
+      // last valid slot of the index row (slots past it are skipped, holes are masked)
+      int last = 0;
+      if (a.idx) {
+        const int32_t* ir = a.idx + qrow * a.topk;
+        for (int k = pt; k < a.topk; k += 64) {
+          const int w = ir[k];
+          if (w >= 0 && w < vis) last = k + 1;
         }
-        rows[e] = row;
-        if (valid) bits |= 1u << e;
+        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+        if (pt == 0) ms->npool_tmp = 0;
+        tc::named_bar_sync(2, 64);
+        if (lane == 0) atomicMax(&ms->npool_tmp, last);
+        tc::named_bar_sync(2, 64);
+        last = ms->npool_tmp;
+      } else {
+        last = vis > 0 ? vis : 0;
       }
-      // gather the 4 bits of every lane into 4 mask words
-      uint32_t word = 0;
-#pragma unroll
-      for (int src = 0; src < 32; ++src) {
-        const uint32_t bb = __shfl_sync(0xffffffffu, bits, src);
-        if ((src >> 3) == (lane & 3)) word |= bb << ((src & 7) * 4);
+      if (pt < R / 2 && (a.rope_q || a.rotate_out)) {
+        double ang = (double)a.qpos[qrow] * P.inv_freq[pt];
+        ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;  // reduce to [-pi, pi]
+        float c, sn;
+        sincosf((float)ang, &sn, &c);
+        d->cs[pt] = c;
+        d->sn[pt] = sn;
       }
-      if (lane < 4) ms->mask[lane] = word;
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive_expect_tx(&ms->kfull, (uint32_t)(nk * D * 2));
-      __syncwarp();
-      if (4 * lane < nk) {
-        const CUtensorMap* mp = pool_grp ? &map_pool : &map_win;
-        uint8_t* dst = smem + L.k + (4 * lane) * 128;
-        for (int c = 0; c < nch; ++c)
-          tc::tma_gather4(dst + c * 16384, mp, c * 64, rows[0], rows[1], rows[2], rows[3], &ms->kfull);
+      if (pt == 0) {
+        d->qrow = qrow;
+        d->t = t;
+        d->vis = vis;
+        d->wlo = wlo;
+        d->nw = nw;
+        d->nw4 = (nw + 3) & ~3;
+        d->npool = last;
+        const int NK = d->nw4 + last;
+        d->ntiles = (NK + kTile - 1) / kTile;
       }
+      tc::named_bar_sync(2, 64);
+      tc::mbar_arrive(&ms->dfull[slot]);
+      // rotate the rope slice of q once it has landed
+      if (!tc::named_bar_and(2, 64, wait_ok(&ms->qfull, n & 1))) {
+        ok = false;
+        break;
+      }
+      if (a.rope_q) {
+        const int npairs = kH * (R / 2);
+        for (int i = pt; i < npairs; i += 64) {
+          const int h = i / (R / 2), k = i % (R / 2);
+          const int dd = rope_lo + 2 * k;
+          uint8_t* p = smem + L.q + (dd / 64) * 8192 + h * 128 + ((((dd % 64) / 8) ^ (h & 7)) * 16) + (dd % 8) * 2;
+          __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(p);
+          const float2 f = __bfloat1622float2(*p2);
+          const float c = d->cs[k], sn = d->sn[k];
+          *p2 = __floats2bfloat162_rn(f.x * c - f.y * sn, f.x * sn + f.y * c);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&ms->qready);
     }
+    if (!ok && pt == 0) atomicExch(&g_attn_tc_error, 6);
+  } else if (warp == 0) {
+    // ================================================================ TMA producer
+    uint32_t g = 0;  // tiles loaded so far (all queries of this CTA)
+    bool ok = true;
+    for (int64_t n = 0; n < nq_cta && ok; ++n) {
+      const int slot = (int)(n & 1);
+      if (!__all_sync(0xffffffffu, wait_ok(&ms->dfull[slot], (n >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      const QDesc* d = &ms->desc[slot];
+      const int64_t qrow = d->qrow;
+      const int b = (int)(qrow / a.Sq);
+      // q of this query, once the previous query's last S^T has read the buffer
+      if (n > 0 && !__all_sync(0xffffffffu, wait_ok(&ms->qfree, (n - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&ms->qfull, (uint32_t)(kH * D * 2));
+        for (int c = 0; c < nch; ++c)
+          tc::tma_load_2d(smem + L.q + c * 8192, &map_q, c * 64, (int)(qrow * kH), &ms->qfull);
+      }
+      const int win_rows = a.win_ring ? a.win_ring : a.kv_rows;
+      const int win_base = b * win_rows;
+      const int pool_base = b * a.P_cap;
+      const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
+      const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
+      const int NK = nw4 + npool;
+      const int ntiles = d->ntiles;
+      for (int i = 0; i < ntiles; ++i, ++g) {
+        const int k0 = i * kTile;
+        const int nvalid = min(kTile, NK - k0);
+        const int nk = (nvalid + 15) & ~15;
+        // rows of this lane's group of 4 keys (masked keys point at a valid row)
+        int rows[4] = {0, 0, 0, 0};
+        const int kg = k0 + 4 * lane;
+        const bool pool_grp = kg >= nw4 && npool > 0;
+        if (4 * lane < nk) {
+          if (pool_grp) {
+            const int p = kg - nw4;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int w = (p + e < npool) ? (ir ? ir[p + e] : p + e) : -1;
+              rows[e] = pool_base + ((w >= 0 && w < vis) ? w : 0);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = kg + e;
+              const int j = k < nw ? wlo + k : wlo;
+              rows[e] = win_base + (a.win_ring ? j % a.win_ring : j);
+            }
+          }
+        }
+        const CUtensorMap* mp = pool_grp ? &map_pool : &map_win;
+        for (int c = 0; c < nch; ++c) {
+          if (g > 0 && !__all_sync(0xffffffffu, wait_ok(&ms->cfree[c], (g - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) tc::mbar_arrive_expect_tx(&ms->cfull[c], (uint32_t)(nk * 128));
+          __syncwarp();
+          if (4 * lane < nk)
+            tc::tma_gather4(smem + L.k + c * 16384 + (4 * lane) * 128, mp, c * 64, rows[0], rows[1], rows[2],
+                            rows[3], &ms->cfull[c]);
+        }
+        if (!ok) break;
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms->dfree[slot]);
+    }
+    if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 1);
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ================================================================ MMA issuer
     const uint32_t idS = tc::idesc_bf16_f32(128, 64, 0, 0);
     const uint32_t idO = tc::idesc_bf16_f32(128, 64, 1, 1);
     const uint32_t kbase = tc::smem_u32(smem + L.k);
     const uint32_t qbase = tc::smem_u32(smem + L.q);
     const uint32_t pbase = tc::smem_u32(smem + L.p);
-    for (int i = 0; i < ntiles; ++i) {
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&ms->kfull, i & 1, kWaitLimit))) {
-        if (lane == 0) set_error(ms, 2);
-        break;
-      }
-      tc::tc_fence_after();
-      const int nvalid = min(kTile, NK - i * kTile);
-      const int nsteps = (nvalid + 15) / 16;
-      if (lane == 0) {
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t ad = tc::sdesc_sw128(kbase + off, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(qbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          tc::umma_f16(tS, ad, bd, idS, kk > 0 ? 1u : 0u);
-        }
-        tc::umma_commit(&ms->sfull);
-      }
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&ms->pfull, i & 1, kWaitLimit))) {
-        if (lane == 0) set_error(ms, 4);
-        break;
-      }
-      tc::tc_fence_after();
-      if (lane == 0) {
-        for (int j = 0; j < nvt; ++j) {
-          for (int kk = 0; kk < nsteps; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(kbase + (2 * j) * 16384 + kk * 2048, 16384, 1024);
-            const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
-            tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        tc::umma_commit(&ms->odone);
-      }
-      __syncwarp();
-    }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue
-    const int q4 = warp & 3;                  // TMEM lane quadrant of this warp
-    const int kk = q4 * 32 + lane;            // key of the tile owned by this thread
-    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const float c1 = a.scale * kLog2e;
-    float l[kH];
-#pragma unroll
-    for (int h = 0; h < kH; ++h) l[h] = 0.f;
-    float sv[kH];
+    uint32_t g = 0;
     bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-      // the 128 softmax threads leave together or not at all (named barriers follow)
-      if (!tc::named_bar_and(1, 128, tc::mbar_wait(&ms->sfull, i & 1, kWaitLimit))) {
-        if (kk == 0) set_error(ms, 5);
+    for (int64_t n = 0; n < nq_cta && ok; ++n) {
+      const int slot = (int)(n & 1);
+      if (!__all_sync(0xffffffffu, wait_ok(&ms->dfull[slot], (n >> 1) & 1))) {
         ok = false;
         break;
       }
-      tc::tc_fence_after();
-      tc::tmem_ld_x64(tS + lane_off, sv);
-      const bool valid = (ms->mask[kk >> 5] >> (kk & 31)) & 1u;
-      bool need = false;
-#pragma unroll
-      for (int h = 0; h < kH; ++h) {
-        sv[h] *= c1;
-        need |= valid && (sv[h] - ms->m[h] > kRescaleThreshold);
+      const QDesc* d = &ms->desc[slot];
+      const int ntiles = d->ntiles;
+      const int NK = d->nw4 + d->npool;
+      if (!__all_sync(0xffffffffu, wait_ok(&ms->qready, n & 1))) {
+        ok = false;
+        break;
       }
-      if (__any_sync(0xffffffffu, need) && lane == 0) atomicAdd(&ms->rescale_cnt[i & 1], 1);
-      tc::named_bar_sync(1, 128);
-      const bool rescale = ms->rescale_cnt[i & 1] != 0;
-      if (tid == kSoftmaxWarp0 * 32) ms->rescale_cnt[(i + 1) & 1] = 0;
-      if (rescale) {
-        // tile max per head over the 128 keys, then raise the running max
+      for (int i = 0; i < ntiles; ++i, ++g) {
+        // S^T = K_tile . Q^T, chunk by chunk as the gathers land
+        for (int c = 0; c < nch; ++c) {
+          if (!__all_sync(0xffffffffu, wait_ok(&ms->cfull[c], g & 1))) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          if (lane == 0) {
 #pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          float v = valid ? sv[h] : -INFINITY;
-          v = warp_max(v);
-          if (lane == 0) ms->red[q4][h] = v;
+            for (int kq = 0; kq < 4; ++kq) {
+              const uint64_t ad = tc::sdesc_sw128(kbase + c * 16384 + kq * 32, 16, 1024);
+              const uint64_t bd = tc::sdesc_sw128(qbase + c * 8192 + kq * 32, 16, 1024);
+              tc::umma_f16(tS, ad, bd, idS, (c > 0 || kq > 0) ? 1u : 0u);
+            }
+          }
+          __syncwarp();
         }
-        tc::named_bar_sync(1, 128);
-        if (tid < kSoftmaxWarp0 * 32 + kH) {
-          const int h = tid - kSoftmaxWarp0 * 32;
-          const float tm = fmaxf(fmaxf(ms->red[0][h], ms->red[1][h]), fmaxf(ms->red[2][h], ms->red[3][h]));
-          const float mo = ms->m[h];
-          const float mn = fmaxf(mo, tm);
-          ms->fac[h] = tc::ex2(mo - mn);
-          ms->m[h] = mn;
+        if (!ok) break;
+        if (lane == 0) {
+          tc::umma_commit(&ms->sfull);
+          // channels that are not values are free once S^T has read them (unless P^T lives there)
+          for (int c = nvch; c < nch; ++c)
+            if (!(alias && c == nch - 1)) tc::umma_commit(&ms->cfree[c]);
+          if (i == ntiles - 1) tc::umma_commit(&ms->qfree);
         }
-        tc::named_bar_sync(1, 128);
-#pragma unroll
-        for (int h = 0; h < kH; ++h) l[h] *= ms->fac[h];
-        if (i > 0) {  // O^T holds tiles 0..i-1 (PV(i-1) completed before this tile was loaded)
-          float o[kH];
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, wait_ok(&ms->pfull, g & 1))) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const int nvalid = min(kTile, NK - i * kTile);
+        const int nsteps = (nvalid + 15) / 16;
+        if (lane == 0) {
           for (int j = 0; j < nvt; ++j) {
-            tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
+            for (int kk = 0; kk < nsteps; ++kk) {
+              const uint64_t ad = tc::sdesc_sw128(kbase + (2 * j) * 16384 + kk * 2048, 16384, 1024);
+              const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
+              tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc::umma_commit(&ms->cfree[2 * j]);
+            tc::umma_commit(&ms->cfree[2 * j + 1]);
+          }
+          if (alias) tc::umma_commit(&ms->cfree[nch - 1]);
+          tc::umma_commit(&ms->odone);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (ntiles == 0 && lane == 0) tc::umma_commit(&ms->qfree);  // q was never read
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms->dfree[slot]);
+    }
+    if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 2);
+  } else {
+    // ================================================================ softmax / epilogue
+    const int q4 = warp & 3;                  // TMEM lane quadrant of this warp
+    const int kk = q4 * 32 + lane;            // key of the tile owned by this thread
+    const int st = tid - 64;                  // 0..127
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float c1 = a.scale * kLog2e;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t n = 0; n < nq_cta && ok; ++n) {
+      const int slot = (int)(n & 1);
+      ok = tc::named_bar_and(1, 128, wait_ok(&ms->dfull[slot], (n >> 1) & 1));
+      if (!ok) break;
+      const QDesc* d = &ms->desc[slot];
+      const int64_t qrow = d->qrow;
+      const int ntiles = d->ntiles, nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis;
+      const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
+      if (st < kH) ms->m[st] = a.sink[st] * kLog2e;
+      tc::named_bar_sync(1, 128);
+      float l[kH];
 #pragma unroll
-            for (int h = 0; h < kH; ++h) o[h] *= ms->fac[h];
-            tc::tmem_st_x64(tO + 64 * j + lane_off, o);
+      for (int h = 0; h < kH; ++h) l[h] = 0.f;
+      for (int i = 0; i < ntiles; ++i, ++g) {
+        // validity of this thread's key (the index read is issued before the wait)
+        const int k = i * kTile + kk;
+        bool valid;
+        if (k < nw4) {
+          valid = k < nw;
+        } else {
+          const int p = k - nw4;
+          if (p < npool) {
+            const int w = ir ? ir[p] : p;
+            valid = w >= 0 && w < vis;
+          } else {
+            valid = false;
           }
         }
-        tc::named_bar_sync(1, 128);
-      }
-      // probabilities -> P^T row `kk` (bf16, 128B-swizzled MN-major B operand)
-      uint8_t* prow = smem + L.p + kk * 128;
+        ok = tc::named_bar_and(1, 128, wait_ok(&ms->sfull, g & 1));
+        if (!ok) break;
+        tc::tc_fence_after();
+        float sv[kH];
+        tc::tmem_ld_x64(tS + lane_off, sv);
+        bool need = false;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int h = u * 8 + 2 * e;
-          const float p0 = valid ? tc::ex2(sv[h] - ms->m[h]) : 0.f;
-          const float p1 = valid ? tc::ex2(sv[h + 1] - ms->m[h + 1]) : 0.f;
-          l[h] += p0;
-          l[h + 1] += p1;
-          __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          w4[e] = *reinterpret_cast<uint32_t*>(&pr);
+        for (int h = 0; h < kH; ++h) {
+          sv[h] *= c1;
+          need |= valid && (sv[h] - ms->m[h] > kRescaleThreshold);
         }
-        *reinterpret_cast<uint4*>(prow + ((u ^ (kk & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        if (__any_sync(0xffffffffu, need) && lane == 0) atomicAdd(&ms->rescale_cnt[g & 1], 1);
+        tc::named_bar_sync(1, 128);
+        const bool rescale = ms->rescale_cnt[g & 1] != 0;
+        if (st == 0) ms->rescale_cnt[(g + 1) & 1] = 0;
+        if (rescale) {
+#pragma unroll
+          for (int h = 0; h < kH; ++h) {
+            const float v = warp_max(valid ? sv[h] : -INFINITY);
+            if (lane == 0) ms->red[q4][h] = v;
+          }
+          tc::named_bar_sync(1, 128);
+          if (st < kH) {
+            const float tm = fmaxf(fmaxf(ms->red[0][st], ms->red[1][st]), fmaxf(ms->red[2][st], ms->red[3][st]));
+            const float mo = ms->m[st];
+            const float mn = fmaxf(mo, tm);
+            ms->fac[st] = tc::ex2(mo - mn);
+            ms->m[st] = mn;
+          }
+          tc::named_bar_sync(1, 128);
+#pragma unroll
+          for (int h = 0; h < kH; ++h) l[h] *= ms->fac[h];
+          if (i > 0) {  // O^T holds tiles 0..i-1; S^T(i) completing implies PV(i-1) completed
+            float o[kH];
+            for (int j = 0; j < nvt; ++j) {
+              tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
+#pragma unroll
+              for (int h = 0; h < kH; ++h) o[h] *= ms->fac[h];
+              tc::tmem_st_x64(tO + 64 * j + lane_off, o);
+            }
+          }
+          tc::named_bar_sync(1, 128);
+        }
+        // probabilities -> P^T row `kk` (bf16, 128B-swizzled MN-major B operand)
+        uint8_t* prow = smem + L.p + kk * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = u * 8 + 2 * e;
+            const float p0 = valid ? tc::ex2(sv[h] - ms->m[h]) : 0.f;
+            const float p1 = valid ? tc::ex2(sv[h + 1] - ms->m[h + 1]) : 0.f;
+            l[h] += p0;
+            l[h + 1] += p1;
+            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+            w4[e] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          *reinterpret_cast<uint4*>(prow + ((u ^ (kk & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->pfull);
       }
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&ms->pfull);
-    }
+      if (!ok) break;
 
-    // ------------------------------------------------------------ epilogue
-    const bool have = ok && ntiles > 0;
-    if (have && !tc::mbar_wait(&ms->odone, (ntiles - 1) & 1, kWaitLimit)) set_error(ms, 6);
-    tc::tc_fence_after();
-    // denominators: per-thread partials -> shared memory (the K tile is free now) -> per head
-    float* lpart = reinterpret_cast<float*>(smem + L.k);  // [128][65], 33 KB
-#pragma unroll
-    for (int h = 0; h < kH; ++h) lpart[kk * 65 + h] = l[h];
-    tc::named_bar_sync(1, 128);
-    if (kk < kH) {
-      float sum = 0.f;
-      for (int r = 0; r < 128; ++r) sum += lpart[r * 65 + kk];
-      const float sink2 = a.sink[kk] * kLog2e;
-      ms->inv_l[kk] = 1.f / (sum + tc::ex2(sink2 - ms->m[kk]));
-    }
-    tc::named_bar_sync(1, 128);
-    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + L.k + 36864);  // [64][dv]
-    const int rope_lo = D - R;
-    for (int j = 0; j < nvt; ++j) {
-      float o[kH];
-      if (have) {
-        tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
-        } else {
-#pragma unroll
-        for (int h = 0; h < kH; ++h) o[h] = 0.f;
-      }
-      const int d = 128 * j + kk;
-      const bool rot = a.rotate_out && d >= rope_lo;
-      float c = 1.f, sn = 0.f;
-      if (rot) {
-        c = ms->cs[(d - rope_lo) >> 1];
-        sn = ms->sn[(d - rope_lo) >> 1];
-      }
+      // ---------------------------------------------------------- epilogue of query n
+      // denominators: reduce the per-thread partial sums over the 128 keys of each head
 #pragma unroll
       for (int h = 0; h < kH; ++h) {
-        float v = o[h] * ms->inv_l[h];
-        const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-        if (rot) v = (d & 1) == 0 ? v * c + other * sn : v * c - other * sn;
-        stage[h * a.dv + d] = __float2bfloat16_rn(v);
+        const float v = warp_sum(l[h]);
+        if (lane == 0) ms->red[q4][h] = v;
       }
+      const bool have = ntiles > 0;
+      if (have) {
+        ok = tc::named_bar_and(1, 128, wait_ok(&ms->odone, (g - 1) & 1));
+        if (!ok) break;
+      } else {
+        tc::named_bar_sync(1, 128);
+      }
+      tc::tc_fence_after();
+      if (st < kH) {
+        const float sum = ms->red[0][st] + ms->red[1][st] + ms->red[2][st] + ms->red[3][st];
+        ms->inv_l[st] = 1.f / (sum + tc::ex2(a.sink[st] * kLog2e - ms->m[st]));
+      }
+      tc::named_bar_sync(1, 128);
+      const int rope_lo = D - a.R;
+      __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.out) + qrow * kH * a.dv;
+      for (int j = 0; j < nvt; ++j) {
+        float o[kH];
+        if (have) {
+          tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
+        } else {
+#pragma unroll
+          for (int h = 0; h < kH; ++h) o[h] = 0.f;
+        }
+        const int dd = 128 * j + kk;
+        const bool rot = a.rotate_out && dd >= rope_lo;
+        float c = 1.f, sn = 0.f;
+        if (rot) {
+          c = d->cs[(dd - rope_lo) >> 1];
+          sn = d->sn[(dd - rope_lo) >> 1];
+        }
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+          float v = o[h] * ms->inv_l[h];
+          const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+          if (rot) v = (dd & 1) == 0 ? v * c + other * sn : v * c - other * sn;
+          og[h * a.dv + dd] = __float2bfloat16_rn(v);
+        }
+      }
+      tc::tc_fence_before();
+      tc::named_bar_sync(1, 128);
+      if (st == 0) tc::mbar_arrive(&ms->dfree[slot]);
     }
-    tc::named_bar_sync(1, 128);
-    uint4* og = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kH * a.dv);
-    const uint4* sg = reinterpret_cast<const uint4*>(stage);
-    for (int i = kk; i < kH * a.dv / 8; i += 128) og[i] = sg[i];
+    if (!ok && st == 0) atomicExch(&g_attn_tc_error, 5);
   }
 
   tc::tc_fence_before();
@@ -442,17 +564,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Rows of D bf16 values; boxes of 64 columns x 1 row with the 128-byte swizzle.
-bool make_row_map(CUtensorMap* m, const void* base, int D, int64_t rows) {
+// Rows of D bf16 values; boxes of 64 columns x box_rows rows with the 128-byte swizzle.
+bool make_row_map(CUtensorMap* m, const void* base, int D, int64_t rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows < 1) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 }  // namespace
@@ -473,31 +602,36 @@ bool attn_tc_supported(const AttnArgs& a, int dtype) {
   if (dtype != DSV4_BF16 || a.H != kH) return false;
   if (a.D % 64 != 0 || a.D < 128 || a.D > 576) return false;
   if (a.dv % 128 != 0 || a.dv > 512 || a.dv > a.D) return false;
-  if (a.D > 512 && a.dv > a.D - 64) return false;
-  if (a.R > 128 || ((a.D - a.R) % 8) != 0) return false;
+  if (a.D > 512 && a.dv > a.D - 64) return false;  // P^T aliases the last K chunk
+  if (a.R > 128 || (a.R & 1) || ((a.D - a.R) % 8) != 0) return false;
   if (!a.pool && a.P_cap > 0) return false;
-  // the epilogue stages the denominators (33 KB) and the output tile in the free K tile
-  if ((a.D / 64) * 16384 < 36864 + 128 * a.dv) return false;
   return encode_fn() != nullptr;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.B * a.Sq;
   if (rows == 0) return cudaSuccess;
-  CUtensorMap mw, mp;
+  CUtensorMap mw, mp, mq;
   const int64_t pool_rows = (int64_t)a.B * (a.P_cap > 0 ? a.P_cap : 1);
   const void* pool_ptr = a.pool ? a.pool : a.kv_win;
-  if (!make_row_map(&mp, pool_ptr, a.D, pool_rows)) return cudaErrorInvalidValue;
+  if (!make_row_map(&mp, pool_ptr, a.D, pool_rows, 1)) return cudaErrorInvalidValue;
   if (a.n_win > 0 && a.kv_win) {
     const int64_t wr = (int64_t)a.B * (a.win_ring ? a.win_ring : a.kv_rows);
-    if (!make_row_map(&mw, a.kv_win, a.D, wr)) return cudaErrorInvalidValue;
+    if (!make_row_map(&mw, a.kv_win, a.D, wr, 1)) return cudaErrorInvalidValue;
   } else {
     mw = mp;  // no window branch: never read
   }
+  if (!make_row_map(&mq, a.q, a.D, rows * kH, kH)) return cudaErrorInvalidValue;
+  TcParams P;
+  P.a = a;
+  P.nrows = rows;
+  for (int k = 0; k < 64; ++k) P.inv_freq[k] = (a.R > 0 && k < a.R / 2) ? pow((double)a.theta, -2.0 * k / a.R) : 0.0;
   const Smem L = smem_layout(a.D);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<(unsigned)rows, kThreads, L.total, st>>>(mw, mp, a);
+  const int nsm = num_sms();
+  const int64_t grid = rows < nsm ? rows : nsm;
+  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mw, mp, mq, P);
   note_launch();
   return cudaGetLastError();
 }

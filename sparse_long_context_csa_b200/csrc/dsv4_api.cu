@@ -165,9 +165,10 @@ uint64_t dsv4_launch_count(void) { return g_launches.load(std::memory_order_rela
 
 dsv4_status dsv4_device_check(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return DSV4_ERR_CUDA;
-  int code = 0;
+  int code = 0, code2 = 0;
   if (take_attn_tc_error(&code) != cudaSuccess) return DSV4_ERR_CUDA;
-  return code ? DSV4_ERR_DEVICE_CHECK : DSV4_OK;
+  if (take_indexer_tc_error(&code2) != cudaSuccess) return DSV4_ERR_CUDA;
+  return (code || code2) ? DSV4_ERR_DEVICE_CHECK : DSV4_OK;
 }
 
 size_t dsv4_workspace_bytes(const dsv4_params* p) {

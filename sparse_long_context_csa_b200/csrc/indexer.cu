@@ -323,8 +323,9 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st
   cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)topk_smem);
   for (int64_t r0 = 0; r0 < rows; r0 += a.rows_per_chunk) {
     const int64_t r1 = r0 + a.rows_per_chunk < rows ? r0 + a.rows_per_chunk : rows;
-    cudaError_t e = dtype == DSV4_BF16 ? launch_scores<__nv_bfloat16>(a, r0, r1, st)
-                                       : launch_scores<float>(a, r0, r1, st);
+    cudaError_t e = indexer_tc_supported(a, dtype) ? launch_indexer_tc_scores(a, r0, r1, st)
+                    : dtype == DSV4_BF16             ? launch_scores<__nv_bfloat16>(a, r0, r1, st)
+                                                     : launch_scores<float>(a, r0, r1, st);
     if (e != cudaSuccess) return e;
     topk_kernel<<<(unsigned)(r1 - r0), kTopkThreads, topk_smem, st>>>(a, r0);
     note_launch();

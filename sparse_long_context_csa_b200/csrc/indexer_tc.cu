@@ -1,0 +1,323 @@
+// Lightning Indexer scores on the sm_100a tensor cores (tcgen05 + TMEM), bf16 inputs.
+//
+// Method: "DeepSeek-V4" doc, "Hybrid attention (§2.3)" CSA item — the Lightning Indexer
+// (eqs. 13-17) scores every query against the compressed indexer-key pool;
+// "DeepSeek-V3.2" doc, DSA item 1 — a low-head-count scorer, per-head weights
+// (`weights_proj`), computed directly in bf16/fp32 since the Hadamard rotation is
+// orthogonal.  Score I[t,w] = sum_h wI[t,h] * relu(qI[t,h] . kI_w).
+//
+// The query x pool-key product is a dense contraction, so it runs on the tensor cores,
+// transposed: D^T[entry, (query, head)] = K_tile[128 x cI] . Qg^T, where Qg holds the
+// (query, head) rows of a group of queries (N = queries x heads <= 256).  A TMEM lane is an
+// entry, so the ReLU, the head weights and the sum over heads are thread-local in the
+// epilogue, and each epilogue thread writes one score per query of the group; rows of 128
+// consecutive entries leave coalesced.
+//
+// Warp roles: 0 = TMA producer (entry tiles, 4-stage ring), 1 = MMA issuer and TMEM owner,
+// 2-5 = epilogue (double-buffered TMEM accumulators).  Tiles past the largest visible
+// entry count of the group are skipped (causality).  Grid: (entry splits, query groups).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace dsv4 {
+
+__device__ int g_indexer_tc_error = 0;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kTileE = 128;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+struct IdxTcParams {
+  IndexerArgs a;
+  int64_t row0, row1;      // rows of this chunk (scores rows are relative to row0)
+  int64_t gid0;            // first query group of this launch
+  int QB;                  // queries per group
+  int Npad;                // QB * nI rounded up to 16
+  int tiles_per_split;     // entry tiles per CTA along grid.x
+};
+
+struct IdxSmem {
+  uint32_t a, b, misc, total;
+};
+
+__host__ __device__ inline IdxSmem idx_smem_layout(int cI, int Npad) {
+  IdxSmem s;
+  const int nch = cI / 64;
+  s.a = 0;                                          // kStages x nch x 16 KB
+  s.b = s.a + kStages * nch * 16384;                // nch x Npad x 128 B
+  s.misc = s.b + nch * ((Npad * 128 + 1023) / 1024) * 1024;
+  s.total = s.misc + 4096;
+  return s;
+}
+
+struct IdxMisc {
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int maxvis;
+  int abort_flag;
+  int vis[256];
+  float w[256];
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap map_pool, const IdxTcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const IndexerArgs& a = P.a;
+  const int cI = a.cI, nI = a.nI, QB = P.QB, Npad = P.Npad;
+  const int lg_nI = 31 - __clz(nI);
+  const int nch = cI / 64;
+  const IdxSmem L = idx_smem_layout(cI, Npad);
+  IdxMisc* ms = reinterpret_cast<IdxMisc*>(smem + L.misc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((tc::smem_u32(smem) & 1023u) != 0) {
+    if (tid == 0) atomicExch(&g_indexer_tc_error, 3);
+    return;
+  }
+
+  // query group -> sequence and rows
+  const int groups_per_seq = (a.Sq + QB - 1) / QB;
+  const int64_t gid = P.gid0 + blockIdx.y;
+  const int b = (int)(gid / groups_per_seq);
+  const int s0 = (int)(gid % groups_per_seq) * QB;
+  const int nq = min(QB, a.Sq - s0);
+  const int64_t rbase = (int64_t)b * a.Sq + s0;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&ms->full[i], 1);
+      tc::mbar_init(&ms->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&ms->tfull[i], 1);
+      tc::mbar_init(&ms->tempty[i], 128);
+    }
+    ms->maxvis = 0;
+    ms->abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ms->tmem_base, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
+    tc::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tc::prefetch_tensormap(&map_pool);
+  __syncthreads();
+  // per-query visibility and head weights
+  for (int q = tid; q < QB; q += kThreads) {
+    int v = 0;
+    const int64_t row = rbase + q;
+    if (q < nq && row >= P.row0 && row < P.row1) {
+      const int t = query_cache_index(a.q_index, row, s0 + q);
+      v = visible_entries(t, a.m, a.P_cap);
+      if (v < 0) v = 0;
+    }
+    ms->vis[q] = v;
+    atomicMax(&ms->maxvis, v);
+  }
+  for (int i = tid; i < QB * nI; i += kThreads) ms->w[i] = (i / nI) < nq ? a.wI[rbase * nI + i] : 0.f;
+  // (query, head) rows -> K-major 128B-swizzled B operand (rows past the group are zero)
+  {
+    const __nv_bfloat16* qI = static_cast<const __nv_bfloat16*>(a.qI);
+    const int per_row = cI / 8;  // 16-byte pieces per row
+    for (int ci = tid; ci < Npad * per_row; ci += kThreads) {
+      const int r = ci / per_row;
+      const int d0 = (ci % per_row) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < nq * nI) v = *reinterpret_cast<const uint4*>(qI + (rbase * nI + r) * cI + d0);
+      const int ch = d0 / 64, u = (d0 % 64) / 8;
+      const uint32_t chunk_bytes = ((Npad * 128 + 1023) / 1024) * 1024;
+      *reinterpret_cast<uint4*>(smem + L.b + ch * chunk_bytes + r * 128 + ((u ^ (r & 7)) * 16)) = v;
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+
+  const int maxvis = ms->maxvis;
+  const int ntile_all = (maxvis + kTileE - 1) / kTileE;
+  const int t_lo = blockIdx.x * P.tiles_per_split;
+  const int t_hi = min(ntile_all, t_lo + P.tiles_per_split);
+  const int ntiles = t_hi > t_lo ? t_hi - t_lo : 0;
+  const uint32_t tmem = ms->tmem_base;
+  const uint32_t b_chunk = ((Npad * 128 + 1023) / 1024) * 1024;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % kStages;
+      const uint32_t ph = (i / kStages) & 1;
+      if (i >= kStages && !__all_sync(0xffffffffu, tc::mbar_wait(&ms->empty[st], ph ^ 1, kWaitLimit))) {
+        if (lane == 0) atomicExch(&g_indexer_tc_error, 1);
+        break;
+      }
+      if (lane == 0) {
+        const int e0 = (t_lo + i) * kTileE;
+        tc::mbar_arrive_expect_tx(&ms->full[st], (uint32_t)(kTileE * cI * 2));
+        for (int c = 0; c < nch; ++c)
+          tc::tma_load_2d(smem + L.a + (st * nch + c) * 16384, &map_pool, c * 64, b * a.P_cap + e0, &ms->full[st]);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc = tc::idesc_bf16_f32(128, Npad, 0, 0);
+    const uint32_t abase = tc::smem_u32(smem + L.a);
+    const uint32_t bbase = tc::smem_u32(smem + L.b);
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % kStages;
+      const int tb = i & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&ms->full[st], (i / kStages) & 1, kWaitLimit))) {
+        if (lane == 0) atomicExch(&g_indexer_tc_error, 2);
+        break;
+      }
+      if (i >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&ms->tempty[tb], ((i >> 1) & 1) ^ 1, kWaitLimit))) {
+        if (lane == 0) atomicExch(&g_indexer_tc_error, 4);
+        break;
+      }
+      tc::tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < cI / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t ad = tc::sdesc_sw128(abase + st * nch * 16384 + off, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(bbase + (kk >> 2) * b_chunk + (kk & 3) * 32, 16, 1024);
+          tc::umma_f16(tmem + tb * Npad, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(&ms->empty[st]);
+        tc::umma_commit(&ms->tfull[tb]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int e = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    for (int i = 0; i < ntiles; ++i) {
+      const int tb = i & 1;
+      if (!tc::named_bar_and(1, 128, tc::mbar_wait(&ms->tfull[tb], (i >> 1) & 1, kWaitLimit))) {
+        if (e == 0) atomicExch(&g_indexer_tc_error, 5);
+        break;
+      }
+      tc::tc_fence_after();
+      const int w = (t_lo + i) * kTileE + e;
+      // 64 accumulator columns at a time, column = q * nI + h (nI is a power of two)
+      float acc[64];
+      float sc = 0.f;
+      for (int c0 = 0; c0 < Npad; c0 += 64) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (c0 + 16 * p < Npad) tc::tmem_ld_x16(tmem + tb * Npad + c0 + 16 * p + lane_off, acc + 16 * p);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int col = c0 + j;
+          const int q = col >> lg_nI, h = col & (nI - 1);
+          if (col < Npad && q < nq) {
+            sc = fmaf(ms->w[col], fmaxf(acc[j], 0.f), sc);
+            if (h == nI - 1) {
+              if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
+              sc = 0.f;
+            }
+          }
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&ms->tempty[tb]);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool indexer_tc_supported(const IndexerArgs& a, int dtype) {
+  if (dtype != DSV4_BF16) return false;
+  if (a.cI != 64 && a.cI != 128) return false;
+  if (a.nI < 1 || a.nI > 64 || (256 % a.nI) != 0) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  IdxTcParams P{};
+  P.a = a;
+  P.row0 = r0;
+  P.row1 = r1;
+  // queries per group: fill N = 256 when the sequence is long enough; decode groups are one query
+  int QB = 256 / a.nI;
+  if (QB > a.Sq) QB = a.Sq;
+  P.QB = QB;
+  P.Npad = ((QB * a.nI + 15) / 16) * 16;
+  const int gps = (a.Sq + QB - 1) / QB;
+  const int64_t g_lo = (r0 / a.Sq) * gps + (r0 % a.Sq) / QB;
+  const int64_t g_hi = ((r1 - 1) / a.Sq) * gps + ((r1 - 1) % a.Sq) / QB + 1;
+  P.gid0 = g_lo;
+  const int64_t ngroups = g_hi - g_lo;
+  const int max_tiles = (a.P_cap + kTileE - 1) / kTileE;
+  // split the entry axis when there are too few query groups to fill the GPU
+  int nsplit = 1;
+  if (ngroups < 2 * 148) nsplit = (int)((2 * 148 + ngroups - 1) / ngroups);
+  if (nsplit > max_tiles) nsplit = max_tiles;
+  P.tiles_per_split = (max_tiles + nsplit - 1) / nsplit;
+  nsplit = (max_tiles + P.tiles_per_split - 1) / P.tiles_per_split;
+
+  CUtensorMap m;
+  EncodeTiledFn fn = encode_fn();
+  cuuint64_t dims[2] = {(cuuint64_t)a.cI, (cuuint64_t)a.B * a.P_cap};
+  cuuint64_t strides[1] = {(cuuint64_t)a.cI * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  if (!fn || fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.poolI), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const IdxSmem L = idx_smem_layout(a.cI, P.Npad);
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)nsplit, (unsigned)ngroups);
+  indexer_tc_kernel<<<grid, kThreads, L.total, st>>>(m, P);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t take_indexer_tc_error(int* code) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_indexer_tc_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_indexer_tc_error, &zero, sizeof(int));
+  }
+  *code = v;
+  return e;
+}
+
+}  // namespace dsv4

@@ -36,6 +36,10 @@ struct IndexerArgs {
   int64_t rows_per_chunk;
 };
 cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st);
+// Tensor-core score kernel (bf16): scores of rows [r0, r1) into a.scores.
+bool indexer_tc_supported(const IndexerArgs& a, int dtype);
+cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st);
+cudaError_t take_indexer_tc_error(int* code);
 // Rows of queries whose scores fit in `bytes` of score workspace.
 int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes);
 // Device address (on the current device) of the fixed score scratch used by
