@@ -10,24 +10,31 @@
 // Design.  A persistent CTA per SM walks its queries; the 64 heads of a query share every
 // key row (MQA).
 //  * Keys of a query = window rows, then the selected pool entries, cut into 128-key tiles.
-//    A producer warp gathers each tile with TMA tile::gather4 (4 arbitrary rows per
-//    instruction) in 64-channel chunks, straight into the 128B-swizzled operand layout.
-//    Every chunk has its own full/free barrier pair, so S^T starts on the first chunk that
-//    lands and the next tile's gathers refill a chunk as soon as PV has read it.
+//    Two producer warps fill a tile chunk by chunk (64 channels) with 16-byte cp.async
+//    copies straight into the 128B-swizzled operand layout.  (Measured on B200: TMA moves
+//    these 128-byte row pieces at its per-request rate, ~7 B/clk per SM for tile::gather4,
+//    and 128-row boxes of contiguous window rows were slower than cp.async as well.)  Every
+//    chunk has its own full/free barrier pair, so S^T starts on the first chunk that lands
+//    and the next tile refills a chunk as soon as PV has read it.
 //  * Scores are computed transposed, S^T[key, head] = K_tile . Q^T (M = 128 keys keeps the
 //    tensor core at full rate; 64 heads alone would be a half-rate M=64 shape), and the same
 //    shared-memory tile is read again as V^T (MN-major) for O^T[dim, head] += V^T . P^T: K=V
 //    costs one gather for both products.
-//  * q (64 heads x D) arrives by TMA in the same swizzled layout as soon as the previous
-//    query's last S^T has read the buffer; two prep warps rotate its rope slice in place and
-//    scan the query's index row while the previous query finishes.
-//  * Softmax warps own one key (TMEM lane) each.  The running max per head starts at the
-//    sink logit and is raised only when a score exceeds it by more than 2^8 (the O^T columns
-//    are then rescaled in TMEM), so a typical tile needs no cross-thread reduction.
+//  * q (64 heads x D) arrives by one TMA burst in the same swizzled layout as soon as the
+//    previous query's last S^T has read the buffer; a prep warp scans the query's index row,
+//    then rotates q's rope slice in place while the previous query finishes.
+//  * Eight softmax warps, two per TMEM lane quadrant: a thread owns one key and 32 heads (two
+//    warps per SM sub-partition hide each other's latencies; measured: splitting the MMAs
+//    into N = 32 halves to overlap them with the softmax was slower than N = 64).  The running
+//    max per head starts at the sink logit and is raised only when a score exceeds it by
+//    more than 2^8 (the O^T columns are then rescaled in TMEM), so a typical tile needs no
+//    cross-thread reduction.
 //  * TMEM: S^T 64 columns, O^T dv/128 tiles x 64 columns.  The epilogue reads O^T, applies
-//    1/denominator and the -qpos rotation, and stores straight to global memory.
-// Warp roles: 0 producer (TMA), 1 MMA issuer + TMEM owner, 2-5 softmax/epilogue,
-//             6-7 query prep (descriptor, RoPE of q).
+//    1/denominator, transposes 8x8 blocks inside lane octets (each lane then holds 8
+//    consecutive channels of one head), applies the -qpos rotation and stores 16 bytes.
+// Warp roles: 0 query prep (descriptor, q load, RoPE of q), 1 MMA issuer + TMEM owner,
+//             2-9 softmax/epilogue (heads 0-31: warps 2-5, heads 32-63: warps 6-9),
+//             10-11 tile producers.
 // Every wait is bounded; a role that gives up records g_attn_tc_error and all roles leave
 // their loops together (warp votes / barrier reductions), free TMEM and return.
 #include <cuda.h>
@@ -45,8 +52,9 @@ __device__ int g_attn_tc_error = 0;  // non-zero: a pipeline wait gave up (the C
 namespace {
 
 constexpr int kH = 64;
+constexpr int kHalf = 32;      // heads per softmax half
 constexpr int kTile = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // 12 warps
 constexpr int kMaxChunks = 9;  // D <= 576
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
@@ -82,11 +90,10 @@ struct QDesc {
 
 struct Misc {
   uint64_t cfull[kMaxChunks], cfree[kMaxChunks];
-  uint64_t qfull, qready, qfree, sfull, pfull, odone;
+  uint64_t qfull, qready, qfree, odone, sfull, pfull;
   uint64_t dfull[2], dfree[2];
   uint32_t tmem_base;
-  int rescale_cnt[2];
-  int npool_tmp;
+  int rescale_cnt[2][2];
   float m[kH];
   float fac[kH];
   float red[4][kH];
@@ -100,8 +107,7 @@ __device__ __forceinline__ bool wait_ok(uint64_t* bar, uint32_t parity) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap map_win, const __grid_constant__ CUtensorMap map_pool,
-                   const __grid_constant__ CUtensorMap map_q, const __grid_constant__ TcParams P) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ TcParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const AttnArgs& a = P.a;
   const int D = a.D;
@@ -121,20 +127,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int c = 0; c < kMaxChunks; ++c) {
-      tc::mbar_init(&ms->cfull[c], 1);
+      tc::mbar_init(&ms->cfull[c], 64);  // one arrival per producer thread
       tc::mbar_init(&ms->cfree[c], 1);
     }
     tc::mbar_init(&ms->qfull, 1);
-    tc::mbar_init(&ms->qready, 64);
+    tc::mbar_init(&ms->qready, 32);
     tc::mbar_init(&ms->qfree, 1);
-    tc::mbar_init(&ms->sfull, 1);
-    tc::mbar_init(&ms->pfull, 128);
     tc::mbar_init(&ms->odone, 1);
+    tc::mbar_init(&ms->sfull, 1);
+    tc::mbar_init(&ms->pfull, 256);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&ms->dfull[i], 64);
-      tc::mbar_init(&ms->dfree[i], 3);
+      tc::mbar_init(&ms->dfull[i], 32);
+      tc::mbar_init(&ms->dfree[i], 4);  // producers, MMA, two softmax halves
     }
-    ms->rescale_cnt[0] = ms->rescale_cnt[1] = 0;
+    for (int i = 0; i < 4; ++i) (&ms->rescale_cnt[0][0])[i] = 0;
     tc::mbar_fence_init();
   }
   if (warp == 1) {
@@ -142,8 +148,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tc::prefetch_tensormap(&map_win);
-    tc::prefetch_tensormap(&map_pool);
     tc::prefetch_tensormap(&map_q);
   }
   tc::tc_fence_before();
@@ -152,16 +156,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ms->tmem_base;
   const uint32_t tS = tmem, tO = tmem + 64;
 
-  if (warp >= 6) {
-    // ================================================================ query prep (64 threads)
-    const int pt = tid - 192;
+  if (warp == 0) {
+    // ================================================================ query prep (1 warp)
     const int R = a.R;
     const int rope_lo = D - R;
     bool ok = true;
     for (int64_t n = 0; n < nq_cta; ++n) {
       const int slot = (int)(n & 1);
       const int64_t qrow = blockIdx.x + n * gridDim.x;
-      if (n >= 2 && !tc::named_bar_and(2, 64, wait_ok(&ms->dfree[slot], ((n >> 1) - 1) & 1))) {
+      if (n >= 2 && !__all_sync(0xffffffffu, wait_ok(&ms->dfree[slot], ((n >> 1) - 1) & 1))) {
         ok = false;
         break;
       }
@@ -177,28 +180,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last = 0;
       if (a.idx) {
         const int32_t* ir = a.idx + qrow * a.topk;
-        for (int k = pt; k < a.topk; k += 64) {
+        for (int k = lane; k < a.topk; k += 32) {
           const int w = ir[k];
           if (w >= 0 && w < vis) last = k + 1;
         }
         for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-        if (pt == 0) ms->npool_tmp = 0;
-        tc::named_bar_sync(2, 64);
-        if (lane == 0) atomicMax(&ms->npool_tmp, last);
-        tc::named_bar_sync(2, 64);
-        last = ms->npool_tmp;
       } else {
         last = vis > 0 ? vis : 0;
       }
-      if (pt < R / 2 && (a.rope_q || a.rotate_out)) {
-        double ang = (double)a.qpos[qrow] * P.inv_freq[pt];
-        ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;  // reduce to [-pi, pi]
-        float c, sn;
-        sincosf((float)ang, &sn, &c);
-        d->cs[pt] = c;
-        d->sn[pt] = sn;
+      if (a.rope_q || a.rotate_out) {
+        for (int k = lane; k < R / 2; k += 32) {
+          double ang = (double)a.qpos[qrow] * P.inv_freq[k];
+          ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;  // reduce to [-pi, pi]
+          float c, sn;
+          sincosf((float)ang, &sn, &c);
+          d->cs[k] = c;
+          d->sn[k] = sn;
+        }
       }
-      if (pt == 0) {
+      if (lane == 0) {
         d->qrow = qrow;
         d->t = t;
         d->vis = vis;
@@ -209,42 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int NK = d->nw4 + last;
         d->ntiles = (NK + kTile - 1) / kTile;
       }
-      tc::named_bar_sync(2, 64);
+      __syncwarp();
       tc::mbar_arrive(&ms->dfull[slot]);
-      // rotate the rope slice of q once it has landed
-      if (!tc::named_bar_and(2, 64, wait_ok(&ms->qfull, n & 1))) {
-        ok = false;
-        break;
-      }
-      if (a.rope_q) {
-        const int npairs = kH * (R / 2);
-        for (int i = pt; i < npairs; i += 64) {
-          const int h = i / (R / 2), k = i % (R / 2);
-          const int dd = rope_lo + 2 * k;
-          uint8_t* p = smem + L.q + (dd / 64) * 8192 + h * 128 + ((((dd % 64) / 8) ^ (h & 7)) * 16) + (dd % 8) * 2;
-          __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(p);
-          const float2 f = __bfloat1622float2(*p2);
-          const float c = d->cs[k], sn = d->sn[k];
-          *p2 = __floats2bfloat162_rn(f.x * c - f.y * sn, f.x * sn + f.y * c);
-        }
-      }
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&ms->qready);
-    }
-    if (!ok && pt == 0) atomicExch(&g_attn_tc_error, 6);
-  } else if (warp == 0) {
-    // ================================================================ TMA producer
-    uint32_t g = 0;  // tiles loaded so far (all queries of this CTA)
-    bool ok = true;
-    for (int64_t n = 0; n < nq_cta && ok; ++n) {
-      const int slot = (int)(n & 1);
-      if (!__all_sync(0xffffffffu, wait_ok(&ms->dfull[slot], (n >> 1) & 1))) {
-        ok = false;
-        break;
-      }
-      const QDesc* d = &ms->desc[slot];
-      const int64_t qrow = d->qrow;
-      const int b = (int)(qrow / a.Sq);
       // q of this query, once the previous query's last S^T has read the buffer
       if (n > 0 && !__all_sync(0xffffffffu, wait_ok(&ms->qfree, (n - 1) & 1))) {
         ok = false;
@@ -255,9 +221,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < nch; ++c)
           tc::tma_load_2d(smem + L.q + c * 8192, &map_q, c * 64, (int)(qrow * kH), &ms->qfull);
       }
+      if (!__all_sync(0xffffffffu, wait_ok(&ms->qfull, n & 1))) {
+        ok = false;
+        break;
+      }
+      // rotate the rope slice of q in place: lane owns pair k, 8 heads per batch
+      if (a.rope_q) {
+        for (int k = lane; k < R / 2; k += 32) {
+          const float c = d->cs[k], sn = d->sn[k];
+          const int dd = rope_lo + 2 * k;
+          const uint32_t col = (dd / 64) * 8192 + (dd % 8) * 2;
+          const int unit = (dd % 64) / 8;
+          for (int h0 = 0; h0 < kH; h0 += 8) {
+            __nv_bfloat162 v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int h = h0 + e;
+              v[e] = *reinterpret_cast<const __nv_bfloat162*>(smem + L.q + col + h * 128 + ((unit ^ (h & 7)) * 16));
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int h = h0 + e;
+              const float2 f = __bfloat1622float2(v[e]);
+              *reinterpret_cast<__nv_bfloat162*>(smem + L.q + col + h * 128 + ((unit ^ (h & 7)) * 16)) =
+                  __floats2bfloat162_rn(f.x * c - f.y * sn, f.x * sn + f.y * c);
+            }
+          }
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&ms->qready);
+    }
+    if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 6);
+  } else if (warp >= 10) {
+    // ================================================================ tile producers (2 warps)
+    // Contiguous tiles (window rows without a ring, or every-entry pools) load as one 128-row
+    // TMA box per chunk; selected entries are gathered with 16-byte cp.async copies straight
+    // into the 128B-swizzled layout: per chunk, thread pt copies 16-byte unit (pt & 7) of
+    // rows (pt >> 3) + 8j, j < 16.
+    const int pt = tid - 320;
+    const int u = pt & 7;
+    uint32_t g = 0;  // tiles loaded so far (all queries of this CTA)
+    bool ok = true;
+    for (int64_t n = 0; n < nq_cta && ok; ++n) {
+      const int slot = (int)(n & 1);
+      if (!tc::named_bar_and(3, 64, wait_ok(&ms->dfull[slot], (n >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      const QDesc* d = &ms->desc[slot];
+      const int64_t qrow = d->qrow;
+      const int b = (int)(qrow / a.Sq);
       const int win_rows = a.win_ring ? a.win_ring : a.kv_rows;
-      const int win_base = b * win_rows;
-      const int pool_base = b * a.P_cap;
+      const __nv_bfloat16* win_base = static_cast<const __nv_bfloat16*>(a.kv_win) + (int64_t)b * win_rows * D;
+      const __nv_bfloat16* pool_base = static_cast<const __nv_bfloat16*>(a.pool) + (int64_t)b * a.P_cap * D;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
       const int NK = nw4 + npool;
@@ -266,48 +283,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = i * kTile;
         const int nvalid = min(kTile, NK - k0);
         const int nk = (nvalid + 15) & ~15;
-        // rows of this lane's group of 4 keys (masked keys point at a valid row)
-        int rows[4] = {0, 0, 0, 0};
-        const int kg = k0 + 4 * lane;
-        const bool pool_grp = kg >= nw4 && npool > 0;
-        if (4 * lane < nk) {
-          if (pool_grp) {
-            const int p = kg - nw4;
+        int srow[16];         // source row of key r = (pt >> 3) + 8j (masked keys read a valid row)
+        uint32_t from_pool = 0;  // bit j: that row is a pool entry (else a window row)
+        {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int w = (p + e < npool) ? (ir ? ir[p + e] : p + e) : -1;
-              rows[e] = pool_base + ((w >= 0 && w < vis) ? w : 0);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = kg + e;
-              const int j = k < nw ? wlo + k : wlo;
-              rows[e] = win_base + (a.win_ring ? j % a.win_ring : j);
+          for (int j = 0; j < 16; ++j) {
+            const int r = (pt >> 3) + 8 * j;
+            const int k = k0 + r;
+            if (k >= nw4 && npool > 0) {
+              const int p = k - nw4;
+              const int w = p < npool ? (ir ? ir[p] : p) : -1;
+              srow[j] = (w >= 0 && w < vis) ? w : 0;
+              from_pool |= 1u << j;
+            } else {
+              const int jj = k < nw ? wlo + k : wlo;
+              srow[j] = a.win_ring ? jj % a.win_ring : jj;
             }
           }
         }
-        const CUtensorMap* mp = pool_grp ? &map_pool : &map_win;
         for (int c = 0; c < nch; ++c) {
-          if (g > 0 && !__all_sync(0xffffffffu, wait_ok(&ms->cfree[c], (g - 1) & 1))) {
+          if (g > 0 && !tc::named_bar_and(3, 64, wait_ok(&ms->cfree[c], (g - 1) & 1))) {
             ok = false;
             break;
           }
-          if (lane == 0) tc::mbar_arrive_expect_tx(&ms->cfull[c], (uint32_t)(nk * 128));
-          __syncwarp();
-          if (4 * lane < nk)
-            tc::tma_gather4(smem + L.k + c * 16384 + (4 * lane) * 128, mp, c * 64, rows[0], rows[1], rows[2],
-                            rows[3], &ms->cfull[c]);
+          uint8_t* cb = smem + L.k + c * 16384;
+          {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int r = (pt >> 3) + 8 * j;
+              const __nv_bfloat16* base = ((from_pool >> j) & 1u) ? pool_base : win_base;
+              if (r < nk) tc::cp_async_16(cb + r * 128 + ((u ^ (r & 7)) * 16), base + (int64_t)srow[j] * D + c * 64 + u * 8);
+            }
+            tc::cp_async_arrive_noinc(&ms->cfull[c]);
+          }
         }
         if (!ok) break;
       }
       if (!ok) break;
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&ms->dfree[slot]);
+      if (pt == 0) tc::mbar_arrive(&ms->dfree[slot]);
     }
-    if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 1);
+    if (!ok && pt == 0) atomicExch(&g_attn_tc_error, 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // Per tile: S^T for heads 0-31, S^T for heads 32-63, PV for heads 0-31, PV for 32-63, so
+    // the tensor core works on one half while the softmax of the other half runs.
     const uint32_t idS = tc::idesc_bf16_f32(128, 64, 0, 0);
     const uint32_t idO = tc::idesc_bf16_f32(128, 64, 1, 1);
     const uint32_t kbase = tc::smem_u32(smem + L.k);
@@ -329,12 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       for (int i = 0; i < ntiles; ++i, ++g) {
-        // S^T = K_tile . Q^T, chunk by chunk as the gathers land
+        // S^T (heads 0-31) chunk by chunk as the copies land
         for (int c = 0; c < nch; ++c) {
           if (!__all_sync(0xffffffffu, wait_ok(&ms->cfull[c], g & 1))) {
             ok = false;
             break;
           }
+          tc::fence_proxy_async_smem();  // cp.async wrote the chunk through the generic proxy
           tc::tc_fence_after();
           if (lane == 0) {
 #pragma unroll
@@ -349,33 +369,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (lane == 0) {
           tc::umma_commit(&ms->sfull);
-          // channels that are not values are free once S^T has read them (unless P^T lives there)
           for (int c = nvch; c < nch; ++c)
             if (!(alias && c == nch - 1)) tc::umma_commit(&ms->cfree[c]);
           if (i == ntiles - 1) tc::umma_commit(&ms->qfree);
         }
         __syncwarp();
-        if (!__all_sync(0xffffffffu, wait_ok(&ms->pfull, g & 1))) {
-          ok = false;
-          break;
-        }
-        tc::tc_fence_after();
         const int nvalid = min(kTile, NK - i * kTile);
         const int nsteps = (nvalid + 15) / 16;
-        if (lane == 0) {
-          for (int j = 0; j < nvt; ++j) {
-            for (int kk = 0; kk < nsteps; ++kk) {
-              const uint64_t ad = tc::sdesc_sw128(kbase + (2 * j) * 16384 + kk * 2048, 16384, 1024);
-              const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
-              tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc::umma_commit(&ms->cfree[2 * j]);
-            tc::umma_commit(&ms->cfree[2 * j + 1]);
+        {
+          if (!__all_sync(0xffffffffu, wait_ok(&ms->pfull, g & 1))) {
+            ok = false;
+            break;
           }
-          if (alias) tc::umma_commit(&ms->cfree[nch - 1]);
-          tc::umma_commit(&ms->odone);
+          tc::tc_fence_after();
+          if (lane == 0) {
+            for (int j = 0; j < nvt; ++j) {
+              for (int kk = 0; kk < nsteps; ++kk) {
+                const uint64_t ad = tc::sdesc_sw128(kbase + (2 * j) * 16384 + kk * 2048, 16384, 1024);
+                const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
+                tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc::umma_commit(&ms->cfree[2 * j]);
+              tc::umma_commit(&ms->cfree[2 * j + 1]);
+            }
+            if (alias) tc::umma_commit(&ms->cfree[nch - 1]);
+            tc::umma_commit(&ms->odone);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        if (!ok) break;
       }
       if (!ok) break;
       if (ntiles == 0 && lane == 0) tc::umma_commit(&ms->qfree);  // q was never read
@@ -385,26 +407,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 2);
   } else {
     // ================================================================ softmax / epilogue
+    // Two halves of 4 warps: half hh owns heads [32hh, 32hh+32); thread = key (TMEM lane).
+    const int hh = (warp - 2) >> 2;
     const int q4 = warp & 3;                  // TMEM lane quadrant of this warp
     const int kk = q4 * 32 + lane;            // key of the tile owned by this thread
-    const int st = tid - 64;                  // 0..127
+    const int st = tid - 64 - 128 * hh;       // 0..127 within the half
+    const int bar_id = 1 + hh;
+    const int h0 = kHalf * hh;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c1 = a.scale * kLog2e;
     uint32_t g = 0;
     bool ok = true;
     for (int64_t n = 0; n < nq_cta && ok; ++n) {
       const int slot = (int)(n & 1);
-      ok = tc::named_bar_and(1, 128, wait_ok(&ms->dfull[slot], (n >> 1) & 1));
+      ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->dfull[slot], (n >> 1) & 1));
       if (!ok) break;
       const QDesc* d = &ms->desc[slot];
       const int64_t qrow = d->qrow;
       const int ntiles = d->ntiles, nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
-      if (st < kH) ms->m[st] = a.sink[st] * kLog2e;
-      tc::named_bar_sync(1, 128);
-      float l[kH];
+      if (st < kHalf) ms->m[h0 + st] = a.sink[h0 + st] * kLog2e;
+      tc::named_bar_sync(bar_id, 128);
+      float l[kHalf];
 #pragma unroll
-      for (int h = 0; h < kH; ++h) l[h] = 0.f;
+      for (int h = 0; h < kHalf; ++h) l[h] = 0.f;
       for (int i = 0; i < ntiles; ++i, ++g) {
         // validity of this thread's key (the index read is issued before the wait)
         const int k = i * kTile + kk;
@@ -420,65 +446,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             valid = false;
           }
         }
-        ok = tc::named_bar_and(1, 128, wait_ok(&ms->sfull, g & 1));
+        ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->sfull, g & 1));
         if (!ok) break;
         tc::tc_fence_after();
-        float sv[kH];
-        tc::tmem_ld_x64(tS + lane_off, sv);
+        float sv[kHalf];
+        tc::tmem_ld_x32(tS + h0 + lane_off, sv);
+        const float* mr = ms->m + h0;  // running max of this half (shared-memory broadcast reads)
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < kH; ++h) {
+        for (int h = 0; h < kHalf; ++h) {
           sv[h] *= c1;
-          need |= valid && (sv[h] - ms->m[h] > kRescaleThreshold);
+          need |= valid && (sv[h] - mr[h] > kRescaleThreshold);
         }
-        if (__any_sync(0xffffffffu, need) && lane == 0) atomicAdd(&ms->rescale_cnt[g & 1], 1);
-        tc::named_bar_sync(1, 128);
-        const bool rescale = ms->rescale_cnt[g & 1] != 0;
-        if (st == 0) ms->rescale_cnt[(g + 1) & 1] = 0;
+        if (__any_sync(0xffffffffu, need) && lane == 0) atomicAdd(&ms->rescale_cnt[hh][g & 1], 1);
+        tc::named_bar_sync(bar_id, 128);
+        const bool rescale = ms->rescale_cnt[hh][g & 1] != 0;
+        if (st == 0) ms->rescale_cnt[hh][(g + 1) & 1] = 0;
         if (rescale) {
 #pragma unroll
-          for (int h = 0; h < kH; ++h) {
+          for (int h = 0; h < kHalf; ++h) {
             const float v = warp_max(valid ? sv[h] : -INFINITY);
-            if (lane == 0) ms->red[q4][h] = v;
+            if (lane == 0) ms->red[q4][h0 + h] = v;
           }
-          tc::named_bar_sync(1, 128);
-          if (st < kH) {
-            const float tm = fmaxf(fmaxf(ms->red[0][st], ms->red[1][st]), fmaxf(ms->red[2][st], ms->red[3][st]));
-            const float mo = ms->m[st];
+          tc::named_bar_sync(bar_id, 128);
+          if (st < kHalf) {
+            const int h = h0 + st;
+            const float tm = fmaxf(fmaxf(ms->red[0][h], ms->red[1][h]), fmaxf(ms->red[2][h], ms->red[3][h]));
+            const float mo = ms->m[h];
             const float mn = fmaxf(mo, tm);
-            ms->fac[st] = tc::ex2(mo - mn);
-            ms->m[st] = mn;
+            ms->fac[h] = tc::ex2(mo - mn);
+            ms->m[h] = mn;
           }
-          tc::named_bar_sync(1, 128);
+          tc::named_bar_sync(bar_id, 128);
 #pragma unroll
-          for (int h = 0; h < kH; ++h) l[h] *= ms->fac[h];
+          for (int h = 0; h < kHalf; ++h) l[h] *= ms->fac[h0 + h];
           if (i > 0) {  // O^T holds tiles 0..i-1; S^T(i) completing implies PV(i-1) completed
-            float o[kH];
+            float o[kHalf];
             for (int j = 0; j < nvt; ++j) {
-              tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
+              tc::tmem_ld_x32(tO + 64 * j + h0 + lane_off, o);
 #pragma unroll
-              for (int h = 0; h < kH; ++h) o[h] *= ms->fac[h];
-              tc::tmem_st_x64(tO + 64 * j + lane_off, o);
+              for (int h = 0; h < kHalf; ++h) o[h] *= ms->fac[h0 + h];
+              tc::tmem_st_x32(tO + 64 * j + h0 + lane_off, o);
             }
           }
-          tc::named_bar_sync(1, 128);
+          tc::named_bar_sync(bar_id, 128);
         }
-        // probabilities -> P^T row `kk` (bf16, 128B-swizzled MN-major B operand)
+        // When P^T shares the buffer of the last key chunk (D > 512), that chunk is still read
+        // by the second half's S^T: the first half waits for it before writing P^T.
+
+        // probabilities -> this half of P^T row `kk` (bf16, 128B-swizzled MN-major B operand)
         uint8_t* prow = smem + L.p + kk * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int uu = 0; uu < 4; ++uu) {
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int h = u * 8 + 2 * e;
-            const float p0 = valid ? tc::ex2(sv[h] - ms->m[h]) : 0.f;
-            const float p1 = valid ? tc::ex2(sv[h + 1] - ms->m[h + 1]) : 0.f;
+            const int h = uu * 8 + 2 * e;
+            const float p0 = valid ? tc::ex2(sv[h] - mr[h]) : 0.f;
+            const float p1 = valid ? tc::ex2(sv[h + 1] - mr[h + 1]) : 0.f;
             l[h] += p0;
             l[h + 1] += p1;
             __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
             w4[e] = *reinterpret_cast<uint32_t*>(&pr);
           }
-          *reinterpret_cast<uint4*>(prow + ((u ^ (kk & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          *reinterpret_cast<uint4*>(prow + (((4 * hh + uu) ^ (kk & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -487,52 +518,97 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue of query n
-      // denominators: reduce the per-thread partial sums over the 128 keys of each head
+      // denominators: halving butterfly over the warp (each lane ends with one head sum),
+      // then the 4 warps of the half meet in shared memory
+      {
 #pragma unroll
-      for (int h = 0; h < kH; ++h) {
-        const float v = warp_sum(l[h]);
-        if (lane == 0) ms->red[q4][h] = v;
+        for (int sft = 16, half = 16; sft >= 1; sft >>= 1, half >>= 1) {
+          const bool up = (lane & sft) != 0;
+#pragma unroll
+          for (int h = 0; h < half; ++h) {
+            const float keep = up ? l[h + half] : l[h];
+            const float send = up ? l[h] : l[h + half];
+            l[h] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+          }
+        }
+        int hb = 0;
+#pragma unroll
+        for (int sft = 16, half = 16; sft >= 1; sft >>= 1, half >>= 1)
+          if (lane & sft) hb += half;
+        ms->red[q4][h0 + hb] = l[0];
       }
       const bool have = ntiles > 0;
       if (have) {
-        ok = tc::named_bar_and(1, 128, wait_ok(&ms->odone, (g - 1) & 1));
+        ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->odone, (g - 1) & 1));
         if (!ok) break;
       } else {
-        tc::named_bar_sync(1, 128);
+        tc::named_bar_sync(bar_id, 128);
       }
       tc::tc_fence_after();
-      if (st < kH) {
-        const float sum = ms->red[0][st] + ms->red[1][st] + ms->red[2][st] + ms->red[3][st];
-        ms->inv_l[st] = 1.f / (sum + tc::ex2(a.sink[st] * kLog2e - ms->m[st]));
+      if (st < kHalf) {
+        const int h = h0 + st;
+        const float sum = ms->red[0][h] + ms->red[1][h] + ms->red[2][h] + ms->red[3][h];
+        ms->inv_l[h] = 1.f / (sum + tc::ex2(a.sink[h] * kLog2e - ms->m[h]));
       }
-      tc::named_bar_sync(1, 128);
+      tc::named_bar_sync(bar_id, 128);
+      // O^T lane = dim, column = head.  An 8x8 butterfly transpose inside each octet of lanes
+      // gives every lane 8 consecutive dims of one head: 16-byte stores, and the rope pairs
+      // (d, d+1) sit in the same lane for the -qpos rotation.
       const int rope_lo = D - a.R;
+      const int oct = lane & 7;
       __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.out) + qrow * kH * a.dv;
+      float il[kHalf];
+#pragma unroll
+      for (int h = 0; h < kHalf; ++h) il[h] = ms->inv_l[h0 + h];
       for (int j = 0; j < nvt; ++j) {
-        float o[kH];
+        float o[kHalf];
         if (have) {
-          tc::tmem_ld_x64(tO + 64 * j + lane_off, o);
+          tc::tmem_ld_x32(tO + 64 * j + h0 + lane_off, o);
         } else {
 #pragma unroll
-          for (int h = 0; h < kH; ++h) o[h] = 0.f;
+          for (int h = 0; h < kHalf; ++h) o[h] = 0.f;
         }
-        const int dd = 128 * j + kk;
-        const bool rot = a.rotate_out && dd >= rope_lo;
-        float c = 1.f, sn = 0.f;
-        if (rot) {
-          c = d->cs[(dd - rope_lo) >> 1];
-          sn = d->sn[(dd - rope_lo) >> 1];
-        }
+        const int d0 = 128 * j + q4 * 32 + (lane & ~7);  // first dim of this octet
 #pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          float v = o[h] * ms->inv_l[h];
-          const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-          if (rot) v = (dd & 1) == 0 ? v * c + other * sn : v * c - other * sn;
-          og[h * a.dv + dd] = __float2bfloat16_rn(v);
+        for (int hb = 0; hb < kHalf / 8; ++hb) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = o[hb * 8 + e] * il[hb * 8 + e];
+#pragma unroll
+          for (int sft = 4; sft >= 1; sft >>= 1) {
+            const bool up = (oct & sft) != 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if ((e & sft) == 0) {
+                const float send = up ? x[e] : x[e | sft];
+                const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
+                if (up) x[e] = recv; else x[e | sft] = recv;
+              }
+            }
+          }
+          // x[e] = head (h0 + hb*8 + oct), dim d0 + e
+          if (a.rotate_out && d0 >= rope_lo) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int kp = (d0 + e - rope_lo) >> 1;
+              const float c = d->cs[kp], sn = d->sn[kp];
+              const float x0 = x[e], x1 = x[e + 1];
+              x[e] = x0 * c + x1 * sn;
+              x[e + 1] = x1 * c - x0 * sn;
+            }
+          }
+          uint4 pk;
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[4], x[5]), b3 = __floats2bfloat162_rn(x[6], x[7]);
+          pk.x = *reinterpret_cast<uint32_t*>(&b0);
+          pk.y = *reinterpret_cast<uint32_t*>(&b1);
+          pk.z = *reinterpret_cast<uint32_t*>(&b2);
+          pk.w = *reinterpret_cast<uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(og + (h0 + hb * 8 + oct) * a.dv + d0) = pk;
         }
       }
       tc::tc_fence_before();
-      tc::named_bar_sync(1, 128);
+      tc::named_bar_sync(bar_id, 128);
       if (st == 0) tc::mbar_arrive(&ms->dfree[slot]);
     }
     if (!ok && st == 0) atomicExch(&g_attn_tc_error, 5);
@@ -611,16 +687,7 @@ bool attn_tc_supported(const AttnArgs& a, int dtype) {
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.B * a.Sq;
   if (rows == 0) return cudaSuccess;
-  CUtensorMap mw, mp, mq;
-  const int64_t pool_rows = (int64_t)a.B * (a.P_cap > 0 ? a.P_cap : 1);
-  const void* pool_ptr = a.pool ? a.pool : a.kv_win;
-  if (!make_row_map(&mp, pool_ptr, a.D, pool_rows, 1)) return cudaErrorInvalidValue;
-  if (a.n_win > 0 && a.kv_win) {
-    const int64_t wr = (int64_t)a.B * (a.win_ring ? a.win_ring : a.kv_rows);
-    if (!make_row_map(&mw, a.kv_win, a.D, wr, 1)) return cudaErrorInvalidValue;
-  } else {
-    mw = mp;  // no window branch: never read
-  }
+  CUtensorMap mq;
   if (!make_row_map(&mq, a.q, a.D, rows * kH, kH)) return cudaErrorInvalidValue;
   TcParams P;
   P.a = a;
@@ -631,7 +698,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int nsm = num_sms();
   const int64_t grid = rows < nsm ? rows : nsm;
-  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mw, mp, mq, P);
+  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mq, P);
   note_launch();
   return cudaGetLastError();
 }
