@@ -10,12 +10,13 @@
 // Design.  A persistent CTA per SM walks its queries; the 64 heads of a query share every
 // key row (MQA).
 //  * Keys of a query = window rows, then the selected pool entries, cut into 128-key tiles.
-//    Two producer warps fill a tile chunk by chunk (64 channels) with 16-byte cp.async
-//    copies straight into the 128B-swizzled operand layout.  (Measured on B200: TMA moves
-//    these 128-byte row pieces at its per-request rate, ~7 B/clk per SM for tile::gather4,
-//    and 128-row boxes of contiguous window rows were slower than cp.async as well.)  Every
-//    chunk has its own full/free barrier pair, so S^T starts on the first chunk that lands
-//    and the next tile refills a chunk as soon as PV has read it.
+//    The eight softmax warps copy a tile themselves, chunk by chunk (64 channels), with
+//    16-byte cp.async copies straight into the 128B-swizzled operand layout, right after
+//    handing the previous tile's probabilities to the MMA: the copies overlap PV.  (Measured
+//    on B200: random 128-byte row pieces move at ~18 B/clk per SM from 2 issuing warps and
+//    ~55 B/clk from 8; TMA tile::gather4 ran at ~7 B/clk, and 128-row TMA boxes of window
+//    rows were slower than cp.async as well.)  Every chunk has its own full/free barrier
+//    pair, so S^T starts on the first chunk that lands.
 //  * Scores are computed transposed, S^T[key, head] = K_tile . Q^T (M = 128 keys keeps the
 //    tensor core at full rate; 64 heads alone would be a half-rate M=64 shape), and the same
 //    shared-memory tile is read again as V^T (MN-major) for O^T[dim, head] += V^T . P^T: K=V
@@ -33,8 +34,7 @@
 //    1/denominator, transposes 8x8 blocks inside lane octets (each lane then holds 8
 //    consecutive channels of one head), applies the -qpos rotation and stores 16 bytes.
 // Warp roles: 0 query prep (descriptor, q load, RoPE of q), 1 MMA issuer + TMEM owner,
-//             2-9 softmax/epilogue (heads 0-31: warps 2-5, heads 32-63: warps 6-9),
-//             10-11 tile producers.
+//             2-9 key copies + softmax/epilogue (heads 0-31: warps 2-5, 32-63: warps 6-9).
 // Every wait is bounded; a role that gives up records g_attn_tc_error and all roles leave
 // their loops together (warp votes / barrier reductions), free TMEM and return.
 #include <cuda.h>
@@ -54,7 +54,7 @@ namespace {
 constexpr int kH = 64;
 constexpr int kHalf = 32;      // heads per softmax half
 constexpr int kTile = 128;
-constexpr int kThreads = 384;  // 12 warps
+constexpr int kThreads = 320;  // 10 warps
 constexpr int kMaxChunks = 9;  // D <= 576
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
@@ -93,6 +93,7 @@ struct Misc {
   uint64_t qfull, qready, qfree, odone, sfull, pfull;
   uint64_t dfull[2], dfree[2];
   uint32_t tmem_base;
+  int abort_flag;
   int rescale_cnt[2][2];
   float m[kH];
   float fac[kH];
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int c = 0; c < kMaxChunks; ++c) {
-      tc::mbar_init(&ms->cfull[c], 64);  // one arrival per producer thread
+      tc::mbar_init(&ms->cfull[c], 256);  // one cp.async arrival per softmax thread
       tc::mbar_init(&ms->cfree[c], 1);
     }
     tc::mbar_init(&ms->qfull, 1);
@@ -138,9 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&ms->pfull, 256);
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&ms->dfull[i], 32);
-      tc::mbar_init(&ms->dfree[i], 4);  // producers, MMA, two softmax halves
+      tc::mbar_init(&ms->dfree[i], 3);  // MMA and the two softmax halves
     }
     for (int i = 0; i < 4; ++i) (&ms->rescale_cnt[0][0])[i] = 0;
+    ms->abort_flag = 0;
     tc::mbar_fence_init();
   }
   if (warp == 1) {
@@ -253,76 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(&ms->qready);
     }
     if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 6);
-  } else if (warp >= 10) {
-    // ================================================================ tile producers (2 warps)
-    // Contiguous tiles (window rows without a ring, or every-entry pools) load as one 128-row
-    // TMA box per chunk; selected entries are gathered with 16-byte cp.async copies straight
-    // into the 128B-swizzled layout: per chunk, thread pt copies 16-byte unit (pt & 7) of
-    // rows (pt >> 3) + 8j, j < 16.
-    const int pt = tid - 320;
-    const int u = pt & 7;
-    uint32_t g = 0;  // tiles loaded so far (all queries of this CTA)
-    bool ok = true;
-    for (int64_t n = 0; n < nq_cta && ok; ++n) {
-      const int slot = (int)(n & 1);
-      if (!tc::named_bar_and(3, 64, wait_ok(&ms->dfull[slot], (n >> 1) & 1))) {
-        ok = false;
-        break;
-      }
-      const QDesc* d = &ms->desc[slot];
-      const int64_t qrow = d->qrow;
-      const int b = (int)(qrow / a.Sq);
-      const int win_rows = a.win_ring ? a.win_ring : a.kv_rows;
-      const __nv_bfloat16* win_base = static_cast<const __nv_bfloat16*>(a.kv_win) + (int64_t)b * win_rows * D;
-      const __nv_bfloat16* pool_base = static_cast<const __nv_bfloat16*>(a.pool) + (int64_t)b * a.P_cap * D;
-      const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
-      const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
-      const int NK = nw4 + npool;
-      const int ntiles = d->ntiles;
-      for (int i = 0; i < ntiles; ++i, ++g) {
-        const int k0 = i * kTile;
-        const int nvalid = min(kTile, NK - k0);
-        const int nk = (nvalid + 15) & ~15;
-        int srow[16];         // source row of key r = (pt >> 3) + 8j (masked keys read a valid row)
-        uint32_t from_pool = 0;  // bit j: that row is a pool entry (else a window row)
-        {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int r = (pt >> 3) + 8 * j;
-            const int k = k0 + r;
-            if (k >= nw4 && npool > 0) {
-              const int p = k - nw4;
-              const int w = p < npool ? (ir ? ir[p] : p) : -1;
-              srow[j] = (w >= 0 && w < vis) ? w : 0;
-              from_pool |= 1u << j;
-            } else {
-              const int jj = k < nw ? wlo + k : wlo;
-              srow[j] = a.win_ring ? jj % a.win_ring : jj;
-            }
-          }
-        }
-        for (int c = 0; c < nch; ++c) {
-          if (g > 0 && !tc::named_bar_and(3, 64, wait_ok(&ms->cfree[c], (g - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          uint8_t* cb = smem + L.k + c * 16384;
-          {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int r = (pt >> 3) + 8 * j;
-              const __nv_bfloat16* base = ((from_pool >> j) & 1u) ? pool_base : win_base;
-              if (r < nk) tc::cp_async_16(cb + r * 128 + ((u ^ (r & 7)) * 16), base + (int64_t)srow[j] * D + c * 64 + u * 8);
-            }
-            tc::cp_async_arrive_noinc(&ms->cfull[c]);
-          }
-        }
-        if (!ok) break;
-      }
-      if (!ok) break;
-      if (pt == 0) tc::mbar_arrive(&ms->dfree[slot]);
-    }
-    if (!ok && pt == 0) atomicExch(&g_attn_tc_error, 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     // Per tile: S^T for heads 0-31, S^T for heads 32-63, PV for heads 0-31, PV for 32-63, so
@@ -406,17 +338,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok && lane == 0) atomicExch(&g_attn_tc_error, 2);
   } else {
-    // ================================================================ softmax / epilogue
+    // ================================================================ copies + softmax / epilogue
     // Two halves of 4 warps: half hh owns heads [32hh, 32hh+32); thread = key (TMEM lane).
+    // The 256 threads also copy the key tiles, one tile ahead: right after handing tile i's
+    // probabilities to the MMA they issue the copies of the next tile (possibly the first
+    // tile of the next query), so the copies overlap PV(i) and the epilogue.
     const int hh = (warp - 2) >> 2;
     const int q4 = warp & 3;                  // TMEM lane quadrant of this warp
     const int kk = q4 * 32 + lane;            // key of the tile owned by this thread
     const int st = tid - 64 - 128 * hh;       // 0..127 within the half
+    const int ct = tid - 64;                  // 0..255 over both halves (copy lanes)
     const int bar_id = 1 + hh;
     const int h0 = kHalf * hh;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c1 = a.scale * kLog2e;
-    uint32_t g = 0;
+
+    // Copy key tile i of query descriptor d as tile number gcopy of this CTA.  Threads wait on
+    // the chunk barriers on their own; a give-up sets abort_flag, checked at the next barrier.
+    auto copy_tile = [&](const QDesc* d, int i, uint32_t gcopy) {
+      const int64_t qrow = d->qrow;
+      const int b = (int)(qrow / a.Sq);
+      const __nv_bfloat16* win_base =
+          static_cast<const __nv_bfloat16*>(a.kv_win) + (int64_t)b * (a.win_ring ? a.win_ring : a.kv_rows) * D;
+      const __nv_bfloat16* pool_base = static_cast<const __nv_bfloat16*>(a.pool) + (int64_t)b * a.P_cap * D;
+      const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
+      const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
+      const int cu = ct & 7;
+      const int k0 = i * kTile;
+      const int nvalid = min(kTile, nw4 + npool - k0);
+      const int nk = (nvalid + 15) & ~15;
+      const __nv_bfloat16* src[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = (ct >> 3) + 32 * j;
+        const int kr = k0 + r;
+        if (kr >= nw4 && npool > 0) {
+          const int p = kr - nw4;
+          const int w = p < npool ? (ir ? ir[p] : p) : -1;
+          src[j] = pool_base + (int64_t)((w >= 0 && w < vis) ? w : 0) * D + cu * 8;
+        } else {
+          const int jj = kr < nw ? wlo + kr : wlo;
+          src[j] = win_base + (int64_t)(a.win_ring ? jj % a.win_ring : jj) * D + cu * 8;
+        }
+      }
+      for (int c = 0; c < nch; ++c) {
+        if (gcopy > 0 && !wait_ok(&ms->cfree[c], (gcopy - 1) & 1)) ms->abort_flag = 1;
+        uint8_t* cb = smem + L.k + c * 16384;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = (ct >> 3) + 32 * j;
+          if (r < nk) tc::cp_async_16(cb + r * 128 + ((cu ^ (r & 7)) * 16), src[j] + c * 64);
+        }
+        tc::cp_async_arrive_noinc(&ms->cfull[c]);
+      }
+    };
+
+    uint32_t g = 0;         // tiles softmaxed so far (all queries of this CTA)
+    bool first_copied = false;  // tile 0 of the current query was copied at the end of the previous one
     bool ok = true;
     for (int64_t n = 0; n < nq_cta && ok; ++n) {
       const int slot = (int)(n & 1);
@@ -426,6 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t qrow = d->qrow;
       const int ntiles = d->ntiles, nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
+      if (!first_copied && ntiles > 0) copy_tile(d, 0, g);
+      first_copied = false;
       if (st < kHalf) ms->m[h0 + st] = a.sink[h0 + st] * kLog2e;
       tc::named_bar_sync(bar_id, 128);
       float l[kHalf];
@@ -446,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             valid = false;
           }
         }
-        ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->sfull, g & 1));
+        ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->sfull, g & 1) && ms->abort_flag == 0);
         if (!ok) break;
         tc::tc_fence_after();
         float sv[kHalf];
@@ -491,9 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::named_bar_sync(bar_id, 128);
         }
-        // When P^T shares the buffer of the last key chunk (D > 512), that chunk is still read
-        // by the second half's S^T: the first half waits for it before writing P^T.
-
         // probabilities -> this half of P^T row `kk` (bf16, 128B-swizzled MN-major B operand)
         uint8_t* prow = smem + L.p + kk * 128;
 #pragma unroll
@@ -514,6 +491,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::mbar_arrive(&ms->pfull);
+        // copies of the next tile: this query's next tile, or the next query's first tile
+        if (i + 1 < ntiles) {
+          copy_tile(d, i + 1, g + 1);
+        } else if (n + 1 < nq_cta) {
+          const int ns = (int)((n + 1) & 1);
+          ok = tc::named_bar_and(bar_id, 128, wait_ok(&ms->dfull[ns], ((n + 1) >> 1) & 1));
+          if (!ok) break;
+          if (ms->desc[ns].ntiles > 0) {
+            copy_tile(&ms->desc[ns], 0, g + 1);
+            first_copied = true;
+          }
+        }
       }
       if (!ok) break;
 
