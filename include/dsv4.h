@@ -163,6 +163,9 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* params, const void* qI,
  *   q_index [B,Sq] int32 or NULL   cache index of each query (NULL: s); with
  *                              win_ring == 0 window tokens at or past S select nothing
  *   out     [B,Sq,H,dv] T
+ *   workspace, ws_bytes   optional: with fewer than 148 queries (decode) and a workspace of at
+ *                              least dsv4_workspace_bytes(params), each query's keys are split
+ *                              over several CTAs whose partial results are merged at the end
  */
 dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* params, const void* q, const void* kv_win,
                                  const void* pool, const int32_t* idx, const float* sink,

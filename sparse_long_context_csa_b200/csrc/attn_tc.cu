@@ -30,6 +30,9 @@
 //    max per head starts at the sink logit and is raised only when a score exceeds it by
 //    more than 2^8 (the O^T columns are then rescaled in TMEM), so a typical tile needs no
 //    cross-thread reduction.
+//  * Few queries (decode): each query's tiles are split over several CTAs, which write
+//    unnormalised partial outputs and softmax statistics to the workspace; a small combine
+//    kernel adds the sink, normalises and rotates.
 //  * TMEM: S^T 64 columns, O^T dv/128 tiles x 64 columns.  The epilogue reads O^T, applies
 //    1/denominator, transposes 8x8 blocks inside lane octets (each lane then holds 8
 //    consecutive channels of one head), applies the -qpos rotation and stores 16 bytes.
@@ -64,6 +67,7 @@ struct TcParams {
   AttnArgs a;
   double inv_freq[64];  // theta^(-2k/R), k < R/2
   int64_t nrows;        // B * Sq queries
+  int64_t nitems;       // work items = queries x key splits
 };
 
 struct Smem {
@@ -83,8 +87,8 @@ __host__ __device__ inline Smem smem_layout(int D) {
 }
 
 struct QDesc {
-  int64_t qrow;
-  int t, vis, wlo, nw, nw4, npool, ntiles;
+  int64_t qrow, item;
+  int t, vis, wlo, nw, nw4, npool, ntiles, tile0;  // this item's tiles: [tile0, tile0 + ntiles)
   float cs[64], sn[64];  // RoPE table at the query position
 };
 
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) atomicExch(&g_attn_tc_error, 3);
     return;
   }
-  const int64_t nq_cta = P.nrows > (int64_t)blockIdx.x ? (P.nrows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t nq_cta = P.nitems > (int64_t)blockIdx.x ? (P.nitems - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (tid == 0) {
     for (int c = 0; c < kMaxChunks; ++c) {
@@ -165,7 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t n = 0; n < nq_cta; ++n) {
       const int slot = (int)(n & 1);
-      const int64_t qrow = blockIdx.x + n * gridDim.x;
+      const int64_t item = blockIdx.x + n * gridDim.x;
+      const int64_t qrow = item / a.nsplit;
+      const int split = (int)(item % a.nsplit);
       if (n >= 2 && !__all_sync(0xffffffffu, wait_ok(&ms->dfree[slot], ((n >> 1) - 1) & 1))) {
         ok = false;
         break;
@@ -202,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 0) {
         d->qrow = qrow;
+        d->item = item;
         d->t = t;
         d->vis = vis;
         d->wlo = wlo;
@@ -209,7 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         d->nw4 = (nw + 3) & ~3;
         d->npool = last;
         const int NK = d->nw4 + last;
-        d->ntiles = (NK + kTile - 1) / kTile;
+        const int nt_all = (NK + kTile - 1) / kTile;
+        const int per = (nt_all + a.nsplit - 1) / a.nsplit;
+        const int lo = min(nt_all, split * per);
+        d->tile0 = lo;
+        d->ntiles = min(nt_all, lo + per) - lo;
       }
       __syncwarp();
       tc::mbar_arrive(&ms->dfull[slot]);
@@ -275,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const QDesc* d = &ms->desc[slot];
       const int ntiles = d->ntiles;
       const int NK = d->nw4 + d->npool;
+      const int tile0 = d->tile0;
       if (!__all_sync(0xffffffffu, wait_ok(&ms->qready, n & 1))) {
         ok = false;
         break;
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i == ntiles - 1) tc::umma_commit(&ms->qfree);
         }
         __syncwarp();
-        const int nvalid = min(kTile, NK - i * kTile);
+        const int nvalid = min(kTile, NK - (tile0 + i) * kTile);
         const int nsteps = (nvalid + 15) / 16;
         {
           if (!__all_sync(0xffffffffu, wait_ok(&ms->pfull, g & 1))) {
@@ -364,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
       const int cu = ct & 7;
-      const int k0 = i * kTile;
+      const int k0 = (d->tile0 + i) * kTile;
       const int nvalid = min(kTile, nw4 + npool - k0);
       const int nk = (nvalid + 15) & ~15;
       const __nv_bfloat16* src[4];
@@ -413,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < kHalf; ++h) l[h] = 0.f;
       for (int i = 0; i < ntiles; ++i, ++g) {
         // validity of this thread's key (the index read is issued before the wait)
-        const int k = i * kTile + kk;
+        const int k = (d->tile0 + i) * kTile + kk;
         bool valid;
         if (k < nw4) {
           valid = k < nw;
@@ -534,6 +546,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::named_bar_sync(bar_id, 128);
       }
       tc::tc_fence_after();
+      if (a.nsplit > 1) {
+        // split over keys: unnormalised O, running max (log2 units) and partial denominator of
+        // this item; the combine kernel adds the sink, normalises and rotates.
+        float* po = a.part + d->item * (int64_t)kH * (a.dv + 2);
+        float* pml = po + (int64_t)kH * a.dv;
+        if (st < kHalf) {
+          const int h = h0 + st;
+          pml[2 * h] = ms->m[h];
+          pml[2 * h + 1] = ms->red[0][h] + ms->red[1][h] + ms->red[2][h] + ms->red[3][h];
+        }
+        const int oct = lane & 7;
+        for (int j = 0; j < nvt; ++j) {
+          float o[kHalf];
+          if (have) {
+            tc::tmem_ld_x32(tO + 64 * j + h0 + lane_off, o);
+          } else {
+#pragma unroll
+            for (int h = 0; h < kHalf; ++h) o[h] = 0.f;
+          }
+          const int d0 = 128 * j + q4 * 32 + (lane & ~7);
+#pragma unroll
+          for (int hb = 0; hb < kHalf / 8; ++hb) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = o[hb * 8 + e];
+#pragma unroll
+            for (int sft = 4; sft >= 1; sft >>= 1) {
+              const bool up = (oct & sft) != 0;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if ((e & sft) == 0) {
+                  const float send = up ? x[e] : x[e | sft];
+                  const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
+                  if (up) x[e] = recv; else x[e | sft] = recv;
+                }
+              }
+            }
+            float* dst = po + (int64_t)(h0 + hb * 8 + oct) * a.dv + d0;
+            *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
+          }
+        }
+        tc::tc_fence_before();
+        tc::named_bar_sync(bar_id, 128);
+        if (st == 0) tc::mbar_arrive(&ms->dfree[slot]);
+        continue;
+      }
       if (st < kHalf) {
         const int h = h0 + st;
         const float sum = ms->red[0][h] + ms->red[1][h] + ms->red[2][h] + ms->red[3][h];
@@ -651,6 +710,54 @@ int num_sms() {
 
 }  // namespace
 
+// Merge the key splits of one (query, head): o = sum_s 2^{m_s - M} O_s / (2^{sink - M} +
+// sum_s 2^{m_s - M} l_s), then the -qpos rotation of the rope slice.  One CTA of dv/4
+// threads per (query, head); thread = 4 consecutive channels.
+__global__ void __launch_bounds__(128) attn_split_combine_kernel(const AttnArgs a, const TcParams P) {
+  const int64_t qrow = blockIdx.x / kH;
+  const int h = blockIdx.x % kH;
+  const int t4 = threadIdx.x;  // channels 4*t4 .. 4*t4+3
+  if (4 * t4 >= a.dv) return;
+  const int64_t stride = (int64_t)kH * (a.dv + 2);
+  const float* base = a.part + qrow * a.nsplit * stride;
+  const float sink2 = a.sink[h] * kLog2e;
+  float M = sink2;
+  for (int sp = 0; sp < a.nsplit; ++sp) M = fmaxf(M, base[sp * stride + (int64_t)kH * a.dv + 2 * h]);
+  float L = tc::ex2(sink2 - M);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp = 0; sp < a.nsplit; ++sp) {
+    const float* ml = base + sp * stride + (int64_t)kH * a.dv + 2 * h;
+    const float w = tc::ex2(ml[0] - M);
+    L += w * ml[1];
+    const float4 v = *reinterpret_cast<const float4*>(base + sp * stride + (int64_t)h * a.dv + 4 * t4);
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
+  }
+  const float inv = 1.f / L;
+  float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const int rope_lo = a.D - a.R;
+  if (a.rotate_out && 4 * t4 >= rope_lo) {
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const int kp = (4 * t4 + e - rope_lo) >> 1;
+      double ang = (double)a.qpos[qrow] * P.inv_freq[kp];
+      ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;
+      float c, sn;
+      sincosf((float)ang, &sn, &c);
+      const float x0 = x[e], x1 = x[e + 1];
+      x[e] = x0 * c + x1 * sn;
+      x[e + 1] = x1 * c - x0 * sn;
+    }
+  }
+  __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&b0);
+  pk.y = *reinterpret_cast<uint32_t*>(&b1);
+  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (qrow * kH + h) * a.dv + 4 * t4) = pk;
+}
+
 cudaError_t take_attn_tc_error(int* code) {
   int v = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_attn_tc_error, sizeof(int));
@@ -680,16 +787,34 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   if (!make_row_map(&mq, a.q, a.D, rows * kH, kH)) return cudaErrorInvalidValue;
   TcParams P;
   P.a = a;
+  if (!P.a.part) P.a.nsplit = 1;
   P.nrows = rows;
+  P.nitems = rows * P.a.nsplit;
   for (int k = 0; k < 64; ++k) P.inv_freq[k] = (a.R > 0 && k < a.R / 2) ? pow((double)a.theta, -2.0 * k / a.R) : 0.0;
   const Smem L = smem_layout(a.D);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   const int nsm = num_sms();
-  const int64_t grid = rows < nsm ? rows : nsm;
+  const int64_t grid = P.nitems < nsm ? P.nitems : nsm;
   attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mq, P);
   note_launch();
+  if (P.a.nsplit > 1) {
+    attn_split_combine_kernel<<<(unsigned)(rows * kH), 128, 0, st>>>(P.a, P);
+    note_launch();
+  }
   return cudaGetLastError();
+}
+
+int attn_splits(int64_t rows) {
+  constexpr int64_t kSplitTarget = 296;  // work items to aim for (two per SM on a 148-SM B200)
+  if (rows <= 0 || rows >= kSplitTarget / 2) return 1;
+  int64_t s = (kSplitTarget + rows - 1) / rows;
+  return (int)(s > 16 ? 16 : s);
+}
+
+size_t attn_split_bytes(int64_t rows, int dv) {
+  const int s = attn_splits(rows);
+  return s > 1 ? (size_t)rows * s * kH * (dv + 2) * sizeof(float) : 0;
 }
 
 }  // namespace dsv4

@@ -114,15 +114,26 @@ dsv4_status run_indexer(const dsv4_params* p, const void* qI, const float* wI, c
 
 dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
                      const int32_t* idx, const float* sink, const int64_t* qpos, const int32_t* q_index,
-                     void* out, void* stream) {
+                     void* out, void* workspace, size_t ws_bytes, void* stream) {
   AttnArgs a{};
   a.B = p->B; a.Sq = p->Sq; a.H = p->H; a.D = p->D; a.R = p->R; a.dv = p->dv; a.n_win = p->n_win;
   a.win_ring = p->win_ring; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk; a.rope_q = p->rope_q;
   a.rotate_out = p->rotate_out; a.kv_rows = p->S; a.scale = p->scale; a.theta = p->rope_theta;
   a.q = q; a.kv_win = kv_win; a.pool = pool; a.idx = idx; a.sink = sink; a.qpos = qpos; a.q_index = q_index;
   a.out = out;
-  if ((int64_t)p->B * p->Sq == 0) return DSV4_OK;
-  if (attn_tc_supported(a, p->dtype)) return from_cuda(launch_attn_tc(a, as_stream(stream)));
+  a.part = nullptr;
+  a.nsplit = 1;
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  if (rows == 0) return DSV4_OK;
+  if (attn_tc_supported(a, p->dtype)) {
+    // few queries: split each query's keys over several CTAs when a workspace is given
+    const size_t need = attn_split_bytes(rows, p->dv);
+    if (need > 0 && workspace && ws_bytes >= need) {
+      a.part = static_cast<float*>(workspace);
+      a.nsplit = attn_splits(rows);
+    }
+    return from_cuda(launch_attn_tc(a, as_stream(stream)));
+  }
   return from_cuda(launch_attn_simt(a, p->dtype, as_stream(stream)));
 }
 
@@ -173,7 +184,9 @@ dsv4_status dsv4_device_check(void* stream) {
 
 size_t dsv4_workspace_bytes(const dsv4_params* p) {
   if (!p || check_common(p) != DSV4_OK) return 0;
-  return align_up(layer_idx_bytes(p)) + align_up(scores_bytes(p));
+  const size_t layer = align_up(layer_idx_bytes(p)) + align_up(scores_bytes(p));
+  const size_t attn = align_up(attn_split_bytes((int64_t)p->B * p->Sq, p->dv));
+  return layer > attn ? layer : attn;  // the attention partials reuse the indexer's scores space
 }
 
 dsv4_status dsv4_compress_kv(const dsv4_params* p, int32_t c, const void* x, const void* z, const float* bias,
@@ -220,13 +233,11 @@ dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* p, const void* q, const void
                                  const int32_t* idx, const float* sink, const int64_t* qpos,
                                  const int32_t* q_index, void* out, void* workspace, size_t ws_bytes,
                                  void* stream) {
-  (void)workspace;
-  (void)ws_bytes;
   dsv4_status st = check_common(p);
   if (st != DSV4_OK) return st;
   if ((st = check_attn(p)) != DSV4_OK) return st;
   if ((st = check_attn_ptrs(p, q, kv_win, pool, idx, sink, qpos, q_index, out)) != DSV4_OK) return st;
-  return run_attn(p, q, kv_win, pool, idx, sink, qpos, q_index, out, stream);
+  return run_attn(p, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace, ws_bytes, stream);
 }
 
 dsv4_status dsv4_csa_layer(const dsv4_params* p, const void* q, const void* kv, const void* z, const float* bias,
@@ -253,7 +264,7 @@ dsv4_status dsv4_csa_layer(const dsv4_params* p, const void* q, const void* kv, 
   if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
   if ((st = run_compress(p, p->cI, kI, zI, biasI, pos, 0, poolI, nullptr, stream)) != DSV4_OK) return st;
   if ((st = run_indexer(p, qI, wI, poolI, nullptr, idx_buf, scores, scores_cap, stream)) != DSV4_OK) return st;
-  return run_attn(p, q, kv_rot, pool, idx_buf, sink, pos, nullptr, out, stream);
+  return run_attn(p, q, kv_rot, pool, idx_buf, sink, pos, nullptr, out, nullptr, 0, stream);
 }
 
 dsv4_status dsv4_hca_layer(const dsv4_params* p, const void* q, const void* kv, const void* z, const float* bias,
@@ -271,7 +282,7 @@ dsv4_status dsv4_hca_layer(const dsv4_params* p, const void* q, const void* kv, 
     if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
   if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
   if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
-  return run_attn(p, q, kv_rot, pool, nullptr, sink, pos, nullptr, out, stream);
+  return run_attn(p, q, kv_rot, pool, nullptr, sink, pos, nullptr, out, nullptr, 0, stream);
 }
 
 }  // extern "C"

@@ -58,7 +58,13 @@ struct AttnArgs {
   const int64_t* qpos;
   const int32_t* q_index;
   void* out;
+  float* part;  // split-over-keys partials (workspace) or nullptr
+  int nsplit;   // key splits per query (1 = no split)
 };
+// Key splits per query used by the tensor-core attention for B*Sq queries (a pure function
+// of the sizes, so that the workspace size is one too), and the workspace it needs.
+int attn_splits(int64_t rows);
+size_t attn_split_bytes(int64_t rows, int dv);
 cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 // Tensor-core (tcgen05) path; returns cudaErrorNotSupported when the shape is not covered.
 bool attn_tc_supported(const AttnArgs& a, int dtype);

@@ -203,7 +203,8 @@ def test_sparse_attention_kernel(lib, name, gains, use_idx):
                               "qpos": x["qpos"], "q_index": x["q_index"]})
     didx = torch.from_numpy(idx).cuda() if use_idx else None
     out = torch.empty((w.B, w.Sq, w.H, w.dv), dtype=harness.torch_dtype(w), device="cuda")
-    abi.dsv4_sparse_mqa_attn(params, d["q"], d["win"], d["pool"], didx, d["sink"], d["qpos"], d["q_index"], out)
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(params), 256), dtype=torch.uint8, device="cuda")
+    abi.dsv4_sparse_mqa_attn(params, d["q"], d["win"], d["pool"], didx, d["sink"], d["qpos"], d["q_index"], out, ws)
     abi.dsv4_device_check()
     rows = [(b, s) for b in range(w.B) for s in (sample_rows(w.Sq, 192, 32) if w.Sq > 1 else [0])]
     ref = O.sparse_mqa_attention(x["q"], c["win"], c["pool"], idx, x["sink"], x["qpos"], x["q_index"],
@@ -212,6 +213,32 @@ def test_sparse_attention_kernel(lib, name, gains, use_idx):
     g = _np(out)
     for b, s in rows:
         assert_max_abs(g[b, s], ref[b, s], ATTN_TOL[w.dtype], f"{name} row {(b, s)}")
+
+
+@pytest.mark.parametrize("B,with_ws", [(3, True), (3, False), (40, True)])
+def test_decode_attention_key_splits(lib, B, with_ws):
+    """Few queries: the keys of each query are split over CTAs and merged (or not, without a
+    workspace); 3 sequences give 16 splits, several of them empty."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, S=20000, P_cap=5000, topk=1024, qindex_spread=500)
+    c = _cache(w, {"q": 256.0})
+    x = _query_inputs(w, {"q": 256.0})
+    idx = synth.strided_selection(w, x["q_index"])
+    params = harness.params_for(w)
+    d = harness.to_device(w, {"q": x["q"], "win": c["win"], "pool": c["pool"], "sink": x["sink"],
+                              "qpos": x["qpos"], "q_index": x["q_index"]})
+    out = torch.empty((w.B, 1, w.H, w.dv), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(params), 256), dtype=torch.uint8, device="cuda") if with_ws else None
+    abi.dsv4_sparse_mqa_attn(params, d["q"], d["win"], d["pool"], torch.from_numpy(idx).cuda(), d["sink"],
+                             d["qpos"], d["q_index"], out, ws)
+    abi.dsv4_device_check()
+    rows = [(b, 0) for b in range(w.B)]
+    ref = O.sparse_mqa_attention(x["q"], c["win"], c["pool"], idx, x["sink"], x["qpos"], x["q_index"],
+                                 n_win=w.n_win, m=w.m, scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rope_q=True,
+                                 rotate_out=w.rotate_out, win_ring=w.win_ring, P_cap=w.P_cap, rows=rows)
+    g = _np(out)
+    for b, s in rows:
+        assert_max_abs(g[b, s], ref[b, s], ATTN_TOL["bf16"], f"decode row {b}")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
