@@ -127,29 +127,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkSmemKeys = 40960;  // keys cached in shared memory (160 KB)
 
-// Exclusive block scan of a 0/1 flag; returns the prefix and writes the block total.
-__device__ __forceinline__ int block_flag_scan(bool f, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, f);
-  const int in_warp = __popc(bal & ((1u << lane) - 1u));
-  if (lane == 0) warp_tot[wid] = __popc(bal);
-  __syncthreads();
-  if (wid == 0) {
-    const int nw = kTopkThreads / 32;
-    int v = lane < nw ? warp_tot[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane < nw) warp_tot[lane] = incl - v;  // exclusive
-    if (lane == 31) *total = incl;
-  }
-  __syncthreads();
-  const int r = warp_tot[wid] + in_warp;
-  __syncthreads();
-  return r;
+__device__ __forceinline__ uint32_t row_key(const uint32_t* keys, const float* sc, bool cached, int i) {
+  return cached ? keys[i] : order_key(sc[i]);
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64_t row0) {
@@ -157,8 +136,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
-  __shared__ int warp_tot[32];
-  __shared__ int s_total;
+  __shared__ int wcnt_gt[kTopkThreads / 32], wcnt_eq[kTopkThreads / 32];
 
   const int64_t row = row0 + blockIdx.x;
   const int s = (int)(row % a.Sq);
@@ -166,7 +144,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
   const int vis = visible_entries(t, a.m, a.P_cap);
   const int K = a.topk;
   int32_t* out = a.idx + row * (int64_t)K;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kTopkThreads / 32;
 
   if (vis <= K) {
     for (int i = tid; i < K; i += kTopkThreads) out[i] = i < vis ? i : -1;
@@ -178,15 +157,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
     for (int i = tid; i < vis; i += kTopkThreads) keys[i] = order_key(sc[i]);
   __syncthreads();
 
+  // Radix select of the K-th largest key, 8 bits per pass.  Lanes that hit the same bin are
+  // merged with match_any before the shared-memory atomic (scores share their top bits).
   uint32_t prefix = 0u, mask = 0u;
   int need = K;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < vis; i += kTopkThreads) {
-      const uint32_t k = cached ? keys[i] : order_key(sc[i]);
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    for (int base = 0; base < vis; base += kTopkThreads) {
+      const int i = base + tid;
+      const bool in = i < vis;
+      const uint32_t k = in ? row_key(keys, sc, cached, i) : 0u;
+      const bool hit = in && (k & mask) == prefix;
+      const uint32_t bin = hit ? (k >> shift) & 255u : 256u;
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (hit && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
     }
     __syncthreads();
     if (tid < 32) {
@@ -222,26 +208,49 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
     prefix = s_prefix;
     need = s_need;
     mask |= 255u << shift;
-    __syncthreads();
   }
-  // prefix = key of the K-th largest score; keep all keys > prefix and the `need`
-  // lowest-index keys == prefix, in ascending entry order.
-  int eq_seen = 0, taken = 0;
-  for (int base = 0; base < vis; base += kTopkThreads) {
-    const int i = base + tid;
-    uint32_t k = 0u;
-    if (i < vis) k = cached ? keys[i] : order_key(sc[i]);
-    const bool gt = i < vis && k > prefix;
-    const bool eq = i < vis && k == prefix;
-    const int eq_rank = eq_seen + block_flag_scan(eq, warp_tot, &s_total);
-    const int eq_tot = s_total;
-    const bool take = gt || (eq && eq_rank < need);
-    const int pos = taken + block_flag_scan(take, warp_tot, &s_total);
-    const int take_tot = s_total;
-    if (take && pos < K) out[pos] = i;
-    eq_seen += eq_tot;
-    taken += take_tot;
-    __syncthreads();
+  // prefix = key of the K-th largest score.  Keep every key > prefix and the `need`
+  // lowest-index keys == prefix, written in ascending entry order: each warp owns a contiguous
+  // segment of the row; per-warp counts, one scan over warps, then ordered writes.
+  const int seg = (vis + kWarps - 1) / kWarps;
+  const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
+  int n_gt = 0, n_eq = 0;
+  for (int i = lo + lane; i < hi; i += 32) {
+    const uint32_t k = row_key(keys, sc, cached, i);
+    n_gt += k > prefix;
+    n_eq += k == prefix;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+  }
+  if (lane == 0) {
+    wcnt_gt[warp] = n_gt;
+    wcnt_eq[warp] = n_eq;
+  }
+  __syncthreads();
+  int gt_before = 0, eq_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += wcnt_gt[w];
+    eq_before += wcnt_eq[w];
+  }
+  // output slot of an entry = (kept entries before it): kept-greater before it plus the kept
+  // ties before it (ties are kept while their rank among ties is below `need`)
+  int pos_gt = gt_before, pos_eq = eq_before;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t k = i < hi ? row_key(keys, sc, cached, i) : 0u;
+    const bool gt = i < hi && k > prefix;
+    const bool eq = i < hi && k == prefix;
+    const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+    const unsigned below = (1u << lane) - 1u;
+    const int my_eq_rank = pos_eq + __popc(beq & below);
+    const int kept_eq_before = min(my_eq_rank, need);
+    const int slot = pos_gt + __popc(bgt & below) + kept_eq_before;
+    if ((gt || (eq && my_eq_rank < need)) && slot < K) out[slot] = i;
+    pos_gt += __popc(bgt);
+    pos_eq += __popc(beq);
   }
 }
 

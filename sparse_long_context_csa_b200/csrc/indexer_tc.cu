@@ -122,19 +122,23 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
     atomicMax(&ms->maxvis, v);
   }
   for (int i = tid; i < QB * nI; i += kThreads) ms->w[i] = (i / nI) < nq ? a.wI[rbase * nI + i] : 0.f;
-  // (query, head) rows -> K-major 128B-swizzled B operand (rows past the group are zero)
+  // (query, head) rows -> K-major 128B-swizzled B operand, by cp.async (rows past the group
+  // are zero-filled with plain stores)
   {
     const __nv_bfloat16* qI = static_cast<const __nv_bfloat16*>(a.qI);
     const int per_row = cI / 8;  // 16-byte pieces per row
+    const uint32_t chunk_bytes = ((Npad * 128 + 1023) / 1024) * 1024;
     for (int ci = tid; ci < Npad * per_row; ci += kThreads) {
       const int r = ci / per_row;
       const int d0 = (ci % per_row) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nq * nI) v = *reinterpret_cast<const uint4*>(qI + (rbase * nI + r) * cI + d0);
       const int ch = d0 / 64, u = (d0 % 64) / 8;
-      const uint32_t chunk_bytes = ((Npad * 128 + 1023) / 1024) * 1024;
-      *reinterpret_cast<uint4*>(smem + L.b + ch * chunk_bytes + r * 128 + ((u ^ (r & 7)) * 16)) = v;
+      uint8_t* dst = smem + L.b + ch * chunk_bytes + r * 128 + ((u ^ (r & 7)) * 16);
+      if (r < nq * nI)
+        tc::cp_async_16(dst, qI + (rbase * nI + r) * cI + d0);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   }
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
@@ -211,6 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
     const int q4 = warp & 3;
     const int e = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    // few columns (decode): weights and visibility live in registers for the whole CTA
+    const bool small = Npad == 16;
+    float wsm[16];
+    int qcol[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      qcol[j] = j >> lg_nI;
+      wsm[j] = (small && qcol[j] < nq) ? ms->w[j] : 0.f;
+    }
     for (int i = 0; i < ntiles; ++i) {
       const int tb = i & 1;
       if (!tc::named_bar_and(1, 128, tc::mbar_wait(&ms->tfull[tb], (i >> 1) & 1, kWaitLimit))) {
@@ -219,18 +232,29 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
       }
       tc::tc_fence_after();
       const int w = (t_lo + i) * kTileE + e;
-      // 64 accumulator columns at a time, column = q * nI + h (nI is a power of two)
-      float acc[64];
+      if (small) {
+        float acc[16];
+        tc::tmem_ld_x16(tmem + tb * Npad + lane_off, acc);
+        for (int q = 0; q < nq; ++q) {
+          float sc = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sc = fmaf(qcol[j] == q ? wsm[j] : 0.f, fmaxf(acc[j], 0.f), sc);
+          if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&ms->tempty[tb]);
+        continue;
+      }
+      // 16 accumulator columns at a time, column = q * nI + h (nI is a power of two)
       float sc = 0.f;
-      for (int c0 = 0; c0 < Npad; c0 += 64) {
+      for (int c0 = 0; c0 < Npad; c0 += 16) {
+        float acc[16];
+        tc::tmem_ld_x16(tmem + tb * Npad + c0 + lane_off, acc);
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
-          if (c0 + 16 * p < Npad) tc::tmem_ld_x16(tmem + tb * Npad + c0 + 16 * p + lane_off, acc + 16 * p);
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const int col = c0 + j;
           const int q = col >> lg_nI, h = col & (nI - 1);
-          if (col < Npad && q < nq) {
+          if (q < nq) {
             sc = fmaf(ms->w[col], fmaxf(acc[j], 0.f), sc);
             if (h == nI - 1) {
               if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
