@@ -41,26 +41,89 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def _visible(w, q_index):
+    t = q_index.reshape(-1).astype(np.int64)
+    return np.minimum((t + 1) // w.m, w.P_cap)
+
+
 def attn_keys_per_query(w, q_index):
     """Keys each query attends: window tokens plus min(topk, visible) pool entries."""
     t = q_index.reshape(-1).astype(np.int64)
     win = np.minimum(w.n_win, t + 1) if w.n_win > 0 else np.zeros_like(t)
-    vis = np.minimum((t + 1) // w.m, w.P_cap)
+    vis = _visible(w, q_index)
     pool = np.minimum(vis, w.topk) if w.kind != "hca" else vis
     return win + pool
 
 
-def attn_flops(w, q_index):
-    """Algorithmic FLOPs of one attention launch: H x keys x (D for QK^T + dv for PV) x 2."""
-    return float(attn_keys_per_query(w, q_index).sum()) * w.H * (w.D + w.dv) * 2.0
+def part_work(w, q_index):
+    """Algorithmic (FLOPs, HBM bytes) of one launch of each part of a step.
 
-
-def attn_bytes(w, q_index):
-    """Algorithmic HBM bytes of one attention launch: q, out, gathered K=V rows, idx."""
+    attention: H x keys x (D + dv) x 2 FLOPs; bytes = q + out + index lists + the K=V rows
+      each sequence needs once (prefill: every rotated token row and pool entry; decode:
+      the gathered rows of its one query).
+    indexer_scores: visible entries x nI x cI x 2 FLOPs; bytes = the indexer pool once per
+      sequence + qI + wI + the fp32 score rows written.
+    topk: no FLOPs; bytes = the fp32 score rows read + the index rows written.
+    compress: bytes = token rows (kv and kI), logits and pools written.
+    """
     e = 2 if w.dtype == "bf16" else 4
     nq = w.B * w.Sq
     keys = float(attn_keys_per_query(w, q_index).sum())
-    return nq * w.H * (w.D + w.dv) * e + keys * w.D * e + (nq * w.topk * 4 if w.topk else 0)
+    vis = _visible(w, q_index).astype(np.float64)
+    if w.kind == "decode":
+        kv_bytes = keys * w.D * e
+    else:
+        kv_bytes = w.B * (w.S + w.P_cap) * w.D * e
+    work = {"attention": (keys * w.H * (w.D + w.dv) * 2.0,
+                          nq * w.H * (w.D + w.dv) * e + kv_bytes + (nq * w.topk * 4 if w.topk else 0))}
+    if w.nI > 0:
+        pool_once = float(w.B) * float(vis.reshape(w.B, -1).max(axis=1).mean()) * w.cI * e
+        work["indexer_scores"] = (vis.sum() * w.nI * w.cI * 2.0,
+                                  pool_once + nq * w.nI * (w.cI * e + 4) + vis.sum() * 4)
+        work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
+    if w.kind != "decode":
+        ch = w.D + (w.cI if w.nI else 0)
+        work["compress"] = (0.0, w.B * w.S * ch * e * 2 + w.B * w.P_cap * ch * e + w.B * w.S * w.D * e)
+    return work
+
+
+def roofline_of(name, flops, nbytes, ms, peaks, peak_src):
+    """Roofline entry of one kernel: bound = the larger of its tensor time and HBM time at
+    the measured peaks; achieved = its algorithmic work / its CUDA-event time."""
+    pk_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    pk_b = peaks["hbm_gbs"]
+    t_tensor = flops / (pk_t * 1e12)
+    t_hbm = nbytes / (pk_b * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / (ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": pk_t, "unit": "TFLOP/s", "frac": ach / pk_t,
+                "kernel": name, "kernel_ms": ms, "algorithmic_flops": flops,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+    ach = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": pk_b, "unit": "GB/s", "frac": ach / pk_b,
+            "kernel": name, "kernel_ms": ms, "algorithmic_bytes": nbytes, "peak_source": f"{peak_src} hbm_gbs"}
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a part's main
+# kernel, from one ncu capture of that kernel on that workload, keyed by the SHA-256 of the
+# kernel's source file when it was captured: once the kernel changes, traffic reads null
+# until it is captured again.  Values: (source file, sha256, bytes per launch).
+NCU_TRAFFIC = {}
+PART_SOURCE = {"attention": "attn_tc.cu", "indexer_scores": "indexer_tc.cu", "topk": "indexer.cu",
+               "compress": "compress.cu"}
+
+
+def ncu_traffic(workload: str, part: str):
+    rec = NCU_TRAFFIC.get((workload, part))
+    if rec is None:
+        return None
+    import hashlib
+    path = os.path.join(ROOT, "sparse_long_context_csa_b200", "csrc", rec[0])
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return rec[2] if sha == rec[1] else None
 
 
 class ClockSampler:
@@ -262,12 +325,13 @@ def main():
     host = synth.make_inputs(w)
     params = harness.params_for(w)
     x = harness.to_device(w, host)
-    o = harness.make_outputs(w, params)
+    o = harness.make_outputs(w, params, scores=True)
     stream = torch.cuda.current_stream()
     q_index = host["q_index"]
+    parts = [p for p in harness.PARTS if p in part_work(w, q_index)]
 
-    def step(ev_pair=None):
-        harness.step_parts(w, params, x, o, stream, attn_events=ev_pair)
+    def step(events=None):
+        harness.step_parts(w, params, x, o, stream, events=events)
 
     # warm-up (also starts the clock sampler and lets it settle)
     sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
@@ -281,8 +345,9 @@ def main():
         step()
         torch.cuda.synchronize()
 
-    # timed region: K steps, device time, attention kernel timed separately
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # timed region: K steps, device time; every part bracketed by its own events
+    evs = [{p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for p in parts}
+           for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
@@ -297,11 +362,11 @@ def main():
     n1 = abi.dsv4_launch_count()
     barrier()
     ms = max_over_ranks(start.elapsed_time(end))
-    attn_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])))
+    part_ms = {p: max_over_ranks(float(np.mean([e[p][0].elapsed_time(e[p][1]) for e in evs]))) for p in parts}
     clocks = sampler.summary(wall0, wall1)
     if args.profile_run:
         if rank == 0:
-            print(json.dumps({"profile_run": True, "ms_per_step": ms / args.steps, "attn_ms": attn_ms}), flush=True)
+            print(json.dumps({"profile_run": True, "ms_per_step": ms / args.steps, "part_ms": part_ms}), flush=True)
         return
 
     # end to end through the layer entry point: pinned host inputs in, output back
@@ -339,18 +404,13 @@ def main():
         e2e_val = world * tokens / (e2e_ms / 1e3)
 
     peaks, peak_src = _peaks()
-    if w.kind == "decode":
-        achieved = attn_bytes(w, q_index) / (attn_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "kernel": "sparse attention", "peak_source": f"{peak_src} hbm_gbs"}
-    else:
-        achieved = attn_flops(w, q_index) / (attn_ms / 1e3) / 1e12
-        pk = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
-                "traffic": None, "kernel": "sparse attention",
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
-    roof["kernel_ms"] = attn_ms
+    work = part_work(w, q_index)
+    dom = max(parts, key=lambda p: part_ms[p])
+    roof = roofline_of(dom, work[dom][0], work[dom][1], part_ms[dom], peaks, peak_src)
+    roof["traffic"] = ncu_traffic(w.name, dom)
+    roof["parts_ms"] = part_ms
+    roof["others"] = {p: {k: v for k, v in roofline_of(p, work[p][0], work[p][1], part_ms[p], peaks, peak_src).items()
+                          if k in ("bound", "achieved", "unit", "frac")} for p in parts if p != dom}
 
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": hib, "scaling": "weak",

@@ -144,6 +144,33 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* params, const void* qI,
                                       void* stream);
 
 /*
+ * The two halves of dsv4_indexer_topk as separate calls, for callers that keep the score
+ * rows (to inspect them, reuse them, or bring their own selection) and for timing each
+ * kernel alone.  Same definitions as dsv4_indexer_topk ([V4] CSA item, Lightning Indexer
+ * eqs. 13-17; [V32] DSA items 1-2).
+ *
+ * dsv4_indexer_scores: scores[b*Sq+s, w] = I[w] for every visible entry w < vis (vis as
+ * above); entries w >= vis of a row are left untouched.
+ *   qI, wI, poolI, q_index  as for dsv4_indexer_topk
+ *   scores  [B*Sq, P_cap] f32, caller-owned, 16-byte aligned
+ *
+ * dsv4_topk_select: idx[b,s,:] = the min(topk, vis) entries w < vis with the highest
+ * scores[b*Sq+s, w], in ascending entry order, then -1 (ties: lower w wins; -0 equals +0;
+ * a NaN ranks above +inf when its sign bit is clear and below -inf when it is set).  Only
+ * entries w < vis of each row are read.  Uses m, P_cap, topk, B, Sq (and S when q_index is
+ * NULL) from params; nI and cI are not read.
+ *   scores  [B*Sq, P_cap] f32
+ *   idx     [B,Sq,topk] int32 out
+ * Both validate on the host (DSV4_ERR_ARG / _SHAPE / _ALIGN) before any launch, allocate
+ * nothing and are asynchronous on `stream`.
+ */
+dsv4_status dsv4_indexer_scores(const dsv4_params* params, const void* qI, const float* wI,
+                                const void* poolI, const int32_t* q_index, float* scores,
+                                void* stream);
+dsv4_status dsv4_topk_select(const dsv4_params* params, const float* scores,
+                             const int32_t* q_index, int32_t* idx, void* stream);
+
+/*
  * Sparse shared-K=V MQA attention with sink ([V4] "Hybrid attention (§2.3)": one KV
  * head read as key and value, partial RoPE, -i output rotation (eq. 26), per-head sink
  * (eq. 27), sliding-window K=V branch concatenated with the compressor entries).

@@ -20,7 +20,8 @@ STATUS = {0: "DSV4_OK", 1: "DSV4_ERR_ARG", 2: "DSV4_ERR_SHAPE", 3: "DSV4_ERR_ALI
 
 EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
-            "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check")
+            "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check", "dsv4_indexer_scores",
+            "dsv4_topk_select")
 
 
 class Dsv4Error(RuntimeError):
@@ -57,6 +58,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_compress_kv.argtypes = [P, i32, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.dsv4_indexer_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.dsv4_indexer_scores.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.dsv4_topk_select.argtypes = [P, vp, vp, vp, vp]
     lib.dsv4_sparse_mqa_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_csa_layer.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.dsv4_hca_layer.argtypes = [P] + [vp] * 10 + [sz, vp]
@@ -69,7 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_device_check.argtypes = [vp]
     lib.dsv4_device_check.restype = ctypes.c_int
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
-               "dsv4_hca_layer", "dsv4_indexer_topk_noalloc"):
+               "dsv4_hca_layer", "dsv4_indexer_topk_noalloc", "dsv4_indexer_scores", "dsv4_topk_select"):
         getattr(lib, fn).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -126,6 +129,18 @@ def dsv4_indexer_topk_noalloc(params, qI, wI, poolI, q_index, idx, stream=None):
     """dsv4_indexer_topk without a workspace: scores go to the library's fixed device scratch."""
     _check("dsv4_indexer_topk_noalloc", load().dsv4_indexer_topk_noalloc(
         ctypes.byref(params), _ptr(qI), _ptr(wI), _ptr(poolI), _ptr(q_index), _ptr(idx), _stream(stream)))
+
+
+def dsv4_indexer_scores(params, qI, wI, poolI, q_index, scores, stream=None):
+    """Lightning Indexer scores only: scores[B*Sq, P_cap] f32 (entries past each row's visible count untouched)."""
+    _check("dsv4_indexer_scores", load().dsv4_indexer_scores(
+        ctypes.byref(params), _ptr(qI), _ptr(wI), _ptr(poolI), _ptr(q_index), _ptr(scores), _stream(stream)))
+
+
+def dsv4_topk_select(params, scores, q_index, idx, stream=None):
+    """Per-query top-k over given score rows: idx[B,Sq,topk] ascending entries, then -1."""
+    _check("dsv4_topk_select", load().dsv4_topk_select(
+        ctypes.byref(params), _ptr(scores), _ptr(q_index), _ptr(idx), _stream(stream)))
 
 
 def dsv4_sparse_mqa_attn(params, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace=None,

@@ -33,9 +33,9 @@
 //  * Few queries (decode): each query's tiles are split over several CTAs, which write
 //    unnormalised partial outputs and softmax statistics to the workspace; a small combine
 //    kernel adds the sink, normalises and rotates.
-//  * TMEM: S^T 64 columns, O^T dv/128 tiles x 64 columns.  The epilogue reads O^T, applies
-//    1/denominator, transposes 8x8 blocks inside lane octets (each lane then holds 8
-//    consecutive channels of one head), applies the -qpos rotation and stores 16 bytes.
+//  * TMEM: S^T 64 columns, O^T dv/128 tiles x 64 columns.  The epilogue reads O^T (lane =
+//    channel), swaps half of its heads with the neighbouring lane so that each lane holds
+//    channel pairs (d, d+1), applies 1/denominator and the -qpos rotation and stores pairs.
 // Warp roles: 0 query prep (descriptor, q load, RoPE of q), 1 MMA issuer + TMEM owner,
 //             2-9 key copies + softmax/epilogue (heads 0-31: warps 2-5, 32-63: warps 6-9).
 // Every wait is bounded; a role that gives up records g_attn_tc_error and all roles leave
@@ -556,7 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           pml[2 * h] = ms->m[h];
           pml[2 * h + 1] = ms->red[0][h] + ms->red[1][h] + ms->red[2][h] + ms->red[3][h];
         }
-        const int oct = lane & 7;
+        const bool odd = (lane & 1) != 0;
+        const int hl = h0 + (odd ? kHalf / 2 : 0);
         for (int j = 0; j < nvt; ++j) {
           float o[kHalf];
           if (have) {
@@ -565,27 +566,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < kHalf; ++h) o[h] = 0.f;
           }
-          const int d0 = 128 * j + q4 * 32 + (lane & ~7);
+          const int dd = 128 * j + q4 * 32 + (lane & ~1);
 #pragma unroll
-          for (int hb = 0; hb < kHalf / 8; ++hb) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = o[hb * 8 + e];
-#pragma unroll
-            for (int sft = 4; sft >= 1; sft >>= 1) {
-              const bool up = (oct & sft) != 0;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if ((e & sft) == 0) {
-                  const float send = up ? x[e] : x[e | sft];
-                  const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
-                  if (up) x[e] = recv; else x[e | sft] = recv;
-                }
-              }
-            }
-            float* dst = po + (int64_t)(h0 + hb * 8 + oct) * a.dv + d0;
-            *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
+          for (int i = 0; i < kHalf / 2; ++i) {
+            const float keep = odd ? o[i + kHalf / 2] : o[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + kHalf / 2], 1);
+            *reinterpret_cast<float2*>(po + (int64_t)(hl + i) * a.dv + dd) =
+                odd ? make_float2(recv, keep) : make_float2(keep, recv);
           }
         }
         tc::tc_fence_before();
@@ -599,15 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ms->inv_l[h] = 1.f / (sum + tc::ex2(a.sink[h] * kLog2e - ms->m[h]));
       }
       tc::named_bar_sync(bar_id, 128);
-      // O^T lane = dim, column = head.  An 8x8 butterfly transpose inside each octet of lanes
-      // gives every lane 8 consecutive dims of one head: 16-byte stores, and the rope pairs
-      // (d, d+1) sit in the same lane for the -qpos rotation.
+      // O^T lane = dim, column = head.  One exchange between neighbouring lanes (dims d, d+1)
+      // leaves the even lane with both dims of heads 0-15 of the half and the odd lane with
+      // both dims of heads 16-31: every store is one (d, d+1) pair (64 contiguous bytes of a
+      // head across the 16 lanes), and the rope pairs sit in one lane for the -qpos rotation.
       const int rope_lo = D - a.R;
-      const int oct = lane & 7;
+      const bool odd = (lane & 1) != 0;
+      const int hl = h0 + (odd ? kHalf / 2 : 0);  // first head this lane stores
       __nv_bfloat16* og = static_cast<__nv_bfloat16*>(a.out) + qrow * kH * a.dv;
-      float il[kHalf];
+      float il[kHalf / 2];
 #pragma unroll
-      for (int h = 0; h < kHalf; ++h) il[h] = ms->inv_l[h0 + h];
+      for (int i = 0; i < kHalf / 2; ++i) il[i] = ms->inv_l[hl + i];
       for (int j = 0; j < nvt; ++j) {
         float o[kHalf];
         if (have) {
@@ -616,43 +605,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < kHalf; ++h) o[h] = 0.f;
         }
-        const int d0 = 128 * j + q4 * 32 + (lane & ~7);  // first dim of this octet
+        const int dd = 128 * j + q4 * 32 + (lane & ~1);  // even dim of this lane's pair
+        const bool rot = a.rotate_out && dd >= rope_lo;
+        float c = 1.f, sn = 0.f;
+        if (rot) {
+          c = d->cs[(dd - rope_lo) >> 1];
+          sn = d->sn[(dd - rope_lo) >> 1];
+        }
 #pragma unroll
-        for (int hb = 0; hb < kHalf / 8; ++hb) {
-          float x[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = o[hb * 8 + e] * il[hb * 8 + e];
-#pragma unroll
-          for (int sft = 4; sft >= 1; sft >>= 1) {
-            const bool up = (oct & sft) != 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if ((e & sft) == 0) {
-                const float send = up ? x[e] : x[e | sft];
-                const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
-                if (up) x[e] = recv; else x[e | sft] = recv;
-              }
-            }
+        for (int i = 0; i < kHalf / 2; ++i) {
+          const float keep = odd ? o[i + kHalf / 2] : o[i];
+          const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[i] : o[i + kHalf / 2], 1);
+          float x0 = (odd ? recv : keep) * il[i];  // dim dd
+          float x1 = (odd ? keep : recv) * il[i];  // dim dd + 1
+          if (rot) {
+            const float r0 = x0 * c + x1 * sn;
+            x1 = x1 * c - x0 * sn;
+            x0 = r0;
           }
-          // x[e] = head (h0 + hb*8 + oct), dim d0 + e
-          if (a.rotate_out && d0 >= rope_lo) {
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const int kp = (d0 + e - rope_lo) >> 1;
-              const float c = d->cs[kp], sn = d->sn[kp];
-              const float x0 = x[e], x1 = x[e + 1];
-              x[e] = x0 * c + x1 * sn;
-              x[e + 1] = x1 * c - x0 * sn;
-            }
-          }
-          uint4 pk;
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[4], x[5]), b3 = __floats2bfloat162_rn(x[6], x[7]);
-          pk.x = *reinterpret_cast<uint32_t*>(&b0);
-          pk.y = *reinterpret_cast<uint32_t*>(&b1);
-          pk.z = *reinterpret_cast<uint32_t*>(&b2);
-          pk.w = *reinterpret_cast<uint32_t*>(&b3);
-          *reinterpret_cast<uint4*>(og + (h0 + hb * 8 + oct) * a.dv + d0) = pk;
+          *reinterpret_cast<__nv_bfloat162*>(og + (int64_t)(hl + i) * a.dv + dd) = __floats2bfloat162_rn(x0, x1);
         }
       }
       tc::tc_fence_before();

@@ -229,6 +229,57 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* p, const void* qI, cons
   return run_indexer(p, qI, wI, poolI, q_index, idx, scratch, (size_t)kNoAllocScoreFloats * sizeof(float), stream);
 }
 
+// Rows of one launch of the split entry points (the score grids' y extents stay below 65536).
+constexpr int64_t kSplitChunkRows = 65535;
+
+dsv4_status dsv4_indexer_scores(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
+                                const int32_t* q_index, float* scores, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if ((st = check_indexer(p)) != DSV4_OK) return st;
+  if (!qI || !wI || !poolI || !scores) return DSV4_ERR_ARG;
+  const void* ptrs[] = {qI, wI, poolI, q_index, scores};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (!q_index && p->Sq > p->S) return DSV4_ERR_SHAPE;
+  IndexerArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.nI = p->nI; a.cI = p->cI; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk;
+  a.qI = qI; a.wI = wI; a.poolI = poolI; a.q_index = q_index;
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  for (int64_t r0 = 0; r0 < rows; r0 += kSplitChunkRows) {
+    const int64_t r1 = r0 + kSplitChunkRows < rows ? r0 + kSplitChunkRows : rows;
+    a.scores = scores + r0 * (int64_t)p->P_cap;
+    a.rows_per_chunk = r1 - r0;
+    const cudaError_t e = launch_indexer_scores(a, p->dtype, r0, r1, as_stream(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return DSV4_OK;
+}
+
+dsv4_status dsv4_topk_select(const dsv4_params* p, const float* scores, const int32_t* q_index, int32_t* idx,
+                             void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if (p->topk < 1 || p->P_cap < 1) return DSV4_ERR_SHAPE;
+  if (!scores || !idx) return DSV4_ERR_ARG;
+  const void* ptrs[] = {scores, q_index, idx};
+  for (const void* x : ptrs)
+    if (x && !aligned16(x)) return DSV4_ERR_ALIGN;
+  if (!q_index && p->Sq > p->S) return DSV4_ERR_SHAPE;
+  IndexerArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.nI = p->nI; a.cI = p->cI; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk;
+  a.q_index = q_index; a.idx = idx;
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  for (int64_t r0 = 0; r0 < rows; r0 += kSplitChunkRows) {
+    const int64_t r1 = r0 + kSplitChunkRows < rows ? r0 + kSplitChunkRows : rows;
+    a.scores = const_cast<float*>(scores) + r0 * (int64_t)p->P_cap;
+    a.rows_per_chunk = r1 - r0;
+    const cudaError_t e = launch_topk(a, r0, r1, as_stream(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return DSV4_OK;
+}
+
 dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
                                  const int32_t* idx, const float* sink, const int64_t* qpos,
                                  const int32_t* q_index, void* out, void* workspace, size_t ws_bytes,

@@ -124,19 +124,76 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-constexpr int kTopkThreads = 512;
-constexpr int kTopkSmemKeys = 40960;  // keys cached in shared memory (160 KB)
+constexpr int kTopkBins = 4096;        // radix digits of 12 bits
+constexpr int kTopkSmemKeys = 40960;   // keys cached in shared memory (160 KB)
 
 __device__ __forceinline__ uint32_t row_key(const uint32_t* keys, const float* sc, bool cached, int i) {
   return cached ? keys[i] : order_key(sc[i]);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64_t row0) {
+// Finds the digit holding the need-th largest key of a histogram (digits scanned from the
+// top): *bin = that digit, *rest = how many keys of it are still needed, *cnt = its count.
+// Thread t owns the descending run of digits [top - BPT + 1, top], top = kTopkBins-1-t*BPT.
+template <int NT>
+__device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* wsum, int* bin, int* rest,
+                                           int* cnt_out) {
+  constexpr int BPT = kTopkBins / NT;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int top = kTopkBins - 1 - tid * BPT;
+  int cnt[BPT];
+  int sum = 0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    cnt[k] = (int)hist[top - k];
+    sum += cnt[k];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < NT / 32 ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += n;
+    }
+    if (lane < NT / 32) wsum[lane] = v;
+  }
+  __syncthreads();
+  incl += warp > 0 ? wsum[warp - 1] : 0;
+  const int excl = incl - sum;
+  if (excl < need && need <= incl) {
+    int run = excl;
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+      if (run < need && need <= run + cnt[k]) {
+        *bin = top - k;
+        *rest = need - run;
+        *cnt_out = cnt[k];
+      }
+      run += cnt[k];
+    }
+  }
+  __syncthreads();
+}
+
+// Per-query top-k by radix select over order-preserving keys: a 12-bit digit histogram
+// while the row is loaded, then 12 and 8 more bits over the keys that still match the
+// selected prefix (skipped once the threshold digit holds exactly the keys still needed).
+// Output: the kept entries in ascending entry order, then -1.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(IndexerArgs a, int64_t row0) {
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_need;
-  __shared__ int wcnt_gt[kTopkThreads / 32], wcnt_eq[kTopkThreads / 32];
+  __shared__ uint32_t hist[kTopkBins];
+  __shared__ int wsum[NT / 32];
+  __shared__ int s_bin, s_rest, s_cnt;
+  __shared__ int wcnt_gt[NT / 32], wcnt_eq[NT / 32];
+  constexpr int kWarps = NT / 32;
 
   const int64_t row = row0 + blockIdx.x;
   const int s = (int)(row % a.Sq);
@@ -145,78 +202,48 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
   const int K = a.topk;
   int32_t* out = a.idx + row * (int64_t)K;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = kTopkThreads / 32;
 
   if (vis <= K) {
-    for (int i = tid; i < K; i += kTopkThreads) out[i] = i < vis ? i : -1;
+    for (int i = tid; i < K; i += NT) out[i] = i < vis ? i : -1;
     return;
   }
   const float* sc = a.scores + (int64_t)blockIdx.x * a.P_cap;
   const bool cached = vis <= kTopkSmemKeys;
-  if (cached)
-    for (int i = tid; i < vis; i += kTopkThreads) keys[i] = order_key(sc[i]);
+  for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
   __syncthreads();
-
-  // Radix select of the K-th largest key, 8 bits per pass.  Lanes that hit the same bin are
-  // merged with match_any before the shared-memory atomic (scores share their top bits).
-  uint32_t prefix = 0u, mask = 0u;
-  int need = K;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0u;
-    __syncthreads();
-    for (int base = 0; base < vis; base += kTopkThreads) {
-      const int i = base + tid;
-      const bool in = i < vis;
-      const uint32_t k = in ? row_key(keys, sc, cached, i) : 0u;
-      const bool hit = in && (k & mask) == prefix;
-      const uint32_t bin = hit ? (k >> shift) & 255u : 256u;
-      const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (hit && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l owns bins 255-8l-7 .. 255-8l (a descending run of 8)
-      const int top = 255 - 8 * tid;
-      int cnt[8];
-      int sum = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        cnt[k] = (int)hist[top - k];
-        sum += cnt[k];
-      }
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += n;
-      }
-      const int excl = incl - sum;
-      if (excl < need && need <= incl) {
-        int run = excl;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (run < need && need <= run + cnt[k]) {
-            s_prefix = prefix | ((uint32_t)(top - k) << shift);
-            s_need = need - run;
-          }
-          run += cnt[k];
-        }
-      }
-    }
-    __syncthreads();
-    prefix = s_prefix;
-    need = s_need;
-    mask |= 255u << shift;
+  for (int i = tid; i < vis; i += NT) {
+    const uint32_t k = order_key(sc[i]);
+    if (cached) keys[i] = k;
+    atomicAdd(&hist[k >> 20], 1u);
   }
-  // prefix = key of the K-th largest score.  Keep every key > prefix and the `need`
-  // lowest-index keys == prefix, written in ascending entry order: each warp owns a contiguous
-  // segment of the row; per-warp counts, one scan over warps, then ordered writes.
+  __syncthreads();
+  find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
+  uint32_t prefix = (uint32_t)s_bin << 20, mask = 0xFFF00000u;
+  int need = s_rest;
+  for (int pass = 1; pass < 3 && s_cnt != need; ++pass) {
+    const int shift = pass == 1 ? 8 : 0;
+    const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
+    for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < vis; i += NT) {
+      const uint32_t k = row_key(keys, sc, cached, i);
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    find_digit<NT>(hist, need, wsum, &s_bin, &s_rest, &s_cnt);
+    prefix |= (uint32_t)s_bin << shift;
+    mask |= dmask << shift;
+    need = s_rest;
+  }
+  // Keep every key whose masked value is above `prefix` and the `need` lowest-index keys
+  // equal to it (all of them when the loop stopped early), in ascending entry order: each
+  // warp owns a contiguous segment of the row; per-warp counts, a scan over warps, then
+  // ordered writes.
   const int seg = (vis + kWarps - 1) / kWarps;
   const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
   int n_gt = 0, n_eq = 0;
   for (int i = lo + lane; i < hi; i += 32) {
-    const uint32_t k = row_key(keys, sc, cached, i);
+    const uint32_t k = row_key(keys, sc, cached, i) & mask;
     n_gt += k > prefix;
     n_eq += k == prefix;
   }
@@ -240,7 +267,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexerArgs a, int64
   int pos_gt = gt_before, pos_eq = eq_before;
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
-    const uint32_t k = i < hi ? row_key(keys, sc, cached, i) : 0u;
+    const uint32_t k = i < hi ? row_key(keys, sc, cached, i) & mask : 0u;
     const bool gt = i < hi && k > prefix;
     const bool eq = i < hi && k == prefix;
     const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
@@ -326,19 +353,34 @@ int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes) {
   return r;
 }
 
+cudaError_t launch_indexer_scores(const IndexerArgs& a, int dtype, int64_t r0, int64_t r1, cudaStream_t st) {
+  return indexer_tc_supported(a, dtype) ? launch_indexer_tc_scores(a, r0, r1, st)
+         : dtype == DSV4_BF16           ? launch_scores<__nv_bfloat16>(a, r0, r1, st)
+                                        : launch_scores<float>(a, r0, r1, st);
+}
+
+cudaError_t launch_topk(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  const size_t smem = (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
+  // long rows: 1024 threads per row; short rows: 256, so that several rows share an SM
+  const bool wide = a.P_cap > 4096;
+  cudaError_t e = wide ? cudaFuncSetAttribute(topk_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                       : cudaFuncSetAttribute(topk_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (wide)
+    topk_kernel<1024><<<(unsigned)(r1 - r0), 1024, smem, st>>>(a, r0);
+  else
+    topk_kernel<256><<<(unsigned)(r1 - r0), 256, smem, st>>>(a, r0);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st) {
   const int64_t rows = (int64_t)a.B * a.Sq;
-  const size_t topk_smem = (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
-  cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)topk_smem);
   for (int64_t r0 = 0; r0 < rows; r0 += a.rows_per_chunk) {
     const int64_t r1 = r0 + a.rows_per_chunk < rows ? r0 + a.rows_per_chunk : rows;
-    cudaError_t e = indexer_tc_supported(a, dtype) ? launch_indexer_tc_scores(a, r0, r1, st)
-                    : dtype == DSV4_BF16             ? launch_scores<__nv_bfloat16>(a, r0, r1, st)
-                                                     : launch_scores<float>(a, r0, r1, st);
+    cudaError_t e = launch_indexer_scores(a, dtype, r0, r1, st);
     if (e != cudaSuccess) return e;
-    topk_kernel<<<(unsigned)(r1 - r0), kTopkThreads, topk_smem, st>>>(a, r0);
-    note_launch();
-    e = cudaGetLastError();
+    e = launch_topk(a, r0, r1, st);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

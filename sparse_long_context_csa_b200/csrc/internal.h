@@ -36,6 +36,10 @@ struct IndexerArgs {
   int64_t rows_per_chunk;
 };
 cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st);
+// The two halves of launch_indexer_topk for query rows [r0, r1): score row r lives at
+// a.scores + (r - r0) * P_cap (entries w < vis written, the rest untouched).
+cudaError_t launch_indexer_scores(const IndexerArgs& a, int dtype, int64_t r0, int64_t r1, cudaStream_t st);
+cudaError_t launch_topk(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st);
 // Tensor-core score kernel (bf16): scores of rows [r0, r1) into a.scores.
 bool indexer_tc_supported(const IndexerArgs& a, int dtype);
 cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st);

@@ -56,7 +56,7 @@ def to_device(w, host: dict, device="cuda", pin=False) -> dict:
     return out
 
 
-def make_outputs(w, params: abi.Dsv4Params, device="cuda") -> dict:
+def make_outputs(w, params: abi.Dsv4Params, device="cuda", scores=False) -> dict:
     dt = torch_dtype(w)
     o = {"out": torch.empty((w.B, w.Sq, w.H, w.dv), dtype=dt, device=device)}
     if w.kind != "decode":
@@ -68,6 +68,8 @@ def make_outputs(w, params: abi.Dsv4Params, device="cuda") -> dict:
         o["idx"] = torch.empty((w.B, w.Sq, w.topk), dtype=torch.int32, device=device)
     ws = abi.dsv4_workspace_bytes(params)
     o["workspace"] = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+    if w.nI > 0 and scores:
+        o["scores"] = torch.empty((w.B * w.Sq, w.P_cap), dtype=torch.float32, device=device)
     return o
 
 
@@ -89,26 +91,42 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
         raise ValueError(w.kind)
 
 
-def step_parts(w, params, x: dict, o: dict, stream=None, attn_events=None) -> None:
-    """The same step as ``step`` issued entry point by entry point, so that a pair of CUDA
-    events (``attn_events``) can bracket the sparse-attention launch on ``stream``."""
+PARTS = ("compress", "indexer_scores", "topk", "attention")
+
+
+def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
+    """The same step as ``step`` issued entry point by entry point, the indexer as its two
+    halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select): the same
+    kernels on the same data.  ``events`` maps names of ``PARTS`` to (start, end) CUDA
+    event pairs recorded on ``stream`` around that part."""
     ws = o["workspace"]
+
+    def mark(name, k):
+        if events is not None and name in events:
+            events[name][k].record(stream)
+
     if w.kind in ("csa", "dsa", "hca"):
+        mark("compress", 0)
         abi.dsv4_compress_kv(params, w.D, x["kv"], x.get("z"), x.get("bias"), x["pos"], 1, o["pool"],
                              o["kv_rot"], stream=stream)
-    if w.kind in ("csa", "dsa"):
-        abi.dsv4_compress_kv(params, w.cI, x["kI"], x.get("zI"), x.get("biasI"), None, 0, o["poolI"], None,
-                             stream=stream)
-        abi.dsv4_indexer_topk(params, x["qI"], x["wI"], o["poolI"], None, o["idx"], ws, stream=stream)
-    elif w.kind == "decode":
-        abi.dsv4_indexer_topk(params, x["qI"], x["wI"], x["poolI"], x["q_index"], o["idx"], ws, stream=stream)
-    if attn_events is not None:
-        attn_events[0].record(stream)
+        if w.kind != "hca":
+            abi.dsv4_compress_kv(params, w.cI, x["kI"], x.get("zI"), x.get("biasI"), None, 0, o["poolI"], None,
+                                 stream=stream)
+        mark("compress", 1)
+    if w.nI > 0:
+        poolI = o["poolI"] if w.kind != "decode" else x["poolI"]
+        q_index = x["q_index"] if w.kind == "decode" else None
+        mark("indexer_scores", 0)
+        abi.dsv4_indexer_scores(params, x["qI"], x["wI"], poolI, q_index, o["scores"], stream=stream)
+        mark("indexer_scores", 1)
+        mark("topk", 0)
+        abi.dsv4_topk_select(params, o["scores"], q_index, o["idx"], stream=stream)
+        mark("topk", 1)
+    mark("attention", 0)
     if w.kind == "decode":
         abi.dsv4_sparse_mqa_attn(params, x["q"], x["win"], x["pool"], o["idx"], x["sink"], x["qpos"],
                                  x["q_index"], o["out"], ws, stream=stream)
     else:
         abi.dsv4_sparse_mqa_attn(params, x["q"], o["kv_rot"], o["pool"], o.get("idx") if w.kind != "hca" else None,
                                  x["sink"], x["pos"], None, o["out"], ws, stream=stream)
-    if attn_events is not None:
-        attn_events[1].record(stream)
+    mark("attention", 1)

@@ -90,6 +90,39 @@ def test_indexer_rejects_bad_arguments(abi):
     assert call(_params(abi), wI=FAKE + 4) == 3
 
 
+def test_split_indexer_calls_reject_bad_arguments(abi):
+    lib = abi.load()
+
+    def scores(p, **over):
+        a = dict(qI=FAKE, wI=FAKE, poolI=FAKE, q_index=None, scores=FAKE)
+        a.update(over)
+        return lib.dsv4_indexer_scores(ctypes.byref(p) if p is not None else None, a["qI"], a["wI"], a["poolI"],
+                                       a["q_index"], a["scores"], None)
+
+    def select(p, **over):
+        a = dict(scores=FAKE, q_index=None, idx=FAKE)
+        a.update(over)
+        return lib.dsv4_topk_select(ctypes.byref(p) if p is not None else None, a["scores"], a["q_index"],
+                                    a["idx"], None)
+
+    assert scores(None) == 1
+    assert scores(_params(abi, nI=3)) == 2
+    assert scores(_params(abi, cI=96)) == 2
+    assert scores(_params(abi), scores=None) == 1
+    assert scores(_params(abi), scores=FAKE + 4) == 3
+    assert scores(_params(abi, Sq=9000)) == 2          # more queries than tokens and no q_index
+    assert scores(_params(abi, dtype=5)) == 4
+    assert select(None) == 1
+    assert select(_params(abi, topk=0)) == 2
+    assert select(_params(abi, P_cap=0)) == 2
+    assert select(_params(abi), idx=None) == 1
+    assert select(_params(abi), scores=FAKE + 8) == 3
+    assert select(_params(abi, Sq=9000)) == 2
+    # empty batches return before any launch
+    assert scores(_params(abi, B=0)) == 0
+    assert select(_params(abi, B=0)) == 0
+
+
 def test_compress_and_layers_reject_bad_arguments(abi):
     lib = abi.load()
     p = _params(abi)

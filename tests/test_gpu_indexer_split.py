@@ -1,0 +1,124 @@
+"""The Lightning Indexer's two halves as separate entry points (dsv4_indexer_scores,
+dsv4_topk_select), against the fp64 oracle.
+
+  scores: every visible entry within the a-priori fp32 accumulation bound of the oracle's
+          fp64 score; entries past a row's visible count are left as they were (checked
+          bit for bit against a sentinel).
+  top-k:  bit-exact.  Both sides rank the SAME fp32 score values (written here, on the
+          host), so the decision is taken in the same precision and every tie is decided
+          by the lower-index rule; the rows are built to be tie-heavy (small integers, +0
+          and -0, +-inf) and to cover the cached (<= 40960 visible) and streamed paths.
+  split = fused: scores + top-k through the two calls equals dsv4_indexer_topk.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import dsv4_oracle as O
+from parity_util import sample_rows, score_error_bound
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = np.float32(-1234.5)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_long_context_csa_b200 import abi, harness
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    abi.load()
+    return abi, harness
+
+
+def _indexer_inputs(w):
+    sp = synth.cache_specs(w)
+    specs = synth.tensor_specs(w)
+    x = {k: synth.reshape(w, k, specs[k].full()) for k in ("qI", "wI")}
+    x["poolI"] = sp["poolI"].full().reshape(w.B, w.P_cap, w.cI)
+    x["q_index"], _ = synth.positions(w)
+    return x
+
+
+@pytest.mark.parametrize("name", ["tiny_csa_f32", "csa_prefill_bf16", "csa_decode_bf16"])
+def test_indexer_scores_kernel(lib, name):
+    abi, harness = lib
+    w = synth.WORKLOADS[name]
+    x = _indexer_inputs(w)
+    params = harness.params_for(w)
+    d = harness.to_device(w, x)
+    scores = torch.full((w.B * w.Sq, w.P_cap), float(SENTINEL), dtype=torch.float32, device="cuda")
+    abi.dsv4_indexer_scores(params, d["qI"], d["wI"], d["poolI"], d["q_index"], scores)
+    abi.dsv4_device_check()
+    g = scores.cpu().numpy()
+    rows = [(b, s) for b in range(w.B) for s in (sample_rows(w.Sq, 96, 16) if w.Sq > 1 else [0])]
+    for b, s in rows:
+        t = int(x["q_index"][b, s])
+        vis = O.visible_entries(t, w.m, w.P_cap)
+        ref = O.indexer_scores_row(x["qI"][b, s], x["wI"][b, s], x["poolI"][b], vis)
+        err = score_error_bound(x["qI"][b, s], x["wI"][b, s], x["poolI"][b][:vis], 0.0)
+        row = g[b * w.Sq + s]
+        bad = np.abs(row[:vis].astype(np.float64) - ref) > err
+        assert not bad.any(), f"{name} row {(b, s)}: {int(bad.sum())} scores outside the fp32 bound"
+        assert (row[vis:] == SENTINEL).all(), f"{name} row {(b, s)}: entries past vis={vis} were written"
+
+
+def _tie_heavy_scores(rng, n_rows, P_cap):
+    """Scores drawn from a few small integers (many exact ties), with +-0 and +-inf planted."""
+    sc = rng.integers(-6, 7, size=(n_rows, P_cap)).astype(np.float32)
+    zeros = rng.random((n_rows, P_cap)) < 0.05
+    sc[zeros] = np.where(rng.random(int(zeros.sum())) < 0.5, np.float32(-0.0), np.float32(0.0))
+    sc[rng.random((n_rows, P_cap)) < 0.001] = np.inf
+    sc[rng.random((n_rows, P_cap)) < 0.001] = -np.inf
+    sc[0, :] = 3.0  # one row of all-equal scores: the lowest indices win
+    return sc
+
+
+@pytest.mark.parametrize("P_cap,topk", [(70001, 2048), (9000, 512), (2100, 2048)])
+def test_topk_select_bit_exact(lib, P_cap, topk):
+    abi, harness = lib
+    # m = 1 so that the visible count of cache index t is t + 1: rows below, at and above
+    # topk, around the 40960-key shared-memory cache, and the full pool.
+    vis_list = sorted({1, topk - 1, topk, topk + 1, min(P_cap, 5000), min(P_cap, 40960),
+                       min(P_cap, 40961), P_cap - 1, P_cap})
+    vis_list = [P_cap] + vis_list  # row 0: all-equal scores over the whole pool
+    B, Sq = 1, len(vis_list)
+    q_index = np.array([[v - 1 for v in vis_list]], dtype=np.int32)
+    rng = np.random.default_rng(20261202)
+    sc = _tie_heavy_scores(rng, Sq, P_cap)
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, Sq=Sq, S=P_cap, m=1, P_cap=P_cap, topk=topk)
+    params = harness.params_for(w)
+    dsc = torch.from_numpy(sc).cuda()
+    dqi = torch.from_numpy(q_index).cuda()
+    idx = torch.full((B, Sq, topk), -7, dtype=torch.int32, device="cuda")
+    abi.dsv4_topk_select(params, dsc, dqi, idx)
+    abi.dsv4_device_check()
+    g = idx.cpu().numpy()[0]
+    for s in range(Sq):
+        t = int(q_index[0, s])
+        vis = O.visible_entries(t, 1, P_cap)
+        ranked, _ = O.topk_select_row(sc[s, :vis], topk)
+        want = np.full(topk, -1, dtype=np.int64)
+        want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
+        assert np.array_equal(g[s].astype(np.int64), want), f"row {s} (vis={vis}) differs from the oracle"
+
+
+@pytest.mark.parametrize("name", ["tiny_csa_f32", "csa_decode_bf16"])
+def test_split_calls_equal_fused_call(lib, name):
+    abi, harness = lib
+    w = synth.WORKLOADS[name]
+    x = _indexer_inputs(w)
+    params = harness.params_for(w)
+    d = harness.to_device(w, x)
+    scores = torch.empty((w.B * w.Sq, w.P_cap), dtype=torch.float32, device="cuda")
+    idx_a = torch.empty((w.B, w.Sq, w.topk), dtype=torch.int32, device="cuda")
+    idx_b = torch.empty_like(idx_a)
+    abi.dsv4_indexer_scores(params, d["qI"], d["wI"], d["poolI"], d["q_index"], scores)
+    abi.dsv4_topk_select(params, scores, d["q_index"], idx_a)
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(params), 256), dtype=torch.uint8, device="cuda")
+    abi.dsv4_indexer_topk(params, d["qI"], d["wI"], d["poolI"], d["q_index"], idx_b, ws)
+    abi.dsv4_device_check()
+    assert torch.equal(idx_a, idx_b)
