@@ -271,6 +271,25 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def reduce_max(v: float, world: int, device: str) -> float:
+    """The maximum of `v` over all ranks (every rank must call it, in the same order)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(kind: str, world: int, tokens_per_rank: int, steps: int, ms_max: float):
+    """Whole-job metric from the slowest rank's time for `steps` steps: decode reports
+    microseconds per step; prefill reports the tokens of all ranks per second."""
+    if kind == "decode":
+        return ms_max / steps * 1e3, "us/step", False
+    return world * tokens_per_rank * steps / (ms_max / 1e3), "tokens/s", True
+
+
 def config_of(w):
     c = {"workload": w.name, "B": w.B, "S": w.S, "Sq": w.Sq, "H": w.H, "head_dim": w.D, "rope_dim": w.R,
          "dv": w.dv, "sliding_window": w.n_win, "m": w.m, "overlap": w.overlap, "pool_cap": w.P_cap}
@@ -315,11 +334,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, "cuda")
 
     abi.load()
     host = synth.make_inputs(w)
@@ -396,12 +411,8 @@ def main():
 
     tokens = w.B * w.Sq
     ms_step = ms / args.steps
-    if w.kind == "decode":
-        value, unit, hib = ms_step * 1e3, "us/step", False
-        e2e_val = e2e_ms * 1e3
-    else:
-        value, unit, hib = world * tokens * args.steps / (ms / 1e3), "tokens/s", True
-        e2e_val = world * tokens / (e2e_ms / 1e3)
+    value, unit, hib = job_value(w.kind, world, tokens, args.steps, ms)
+    e2e_val = job_value(w.kind, world, tokens, 1, e2e_ms)[0]
 
     peaks, peak_src = _peaks()
     work = part_work(w, q_index)

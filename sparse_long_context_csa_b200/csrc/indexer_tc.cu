@@ -35,7 +35,7 @@ constexpr int kThreads = 288;  // 4 producer warps, 1 MMA warp, 4 epilogue warps
 constexpr int kProducers = 128;
 constexpr int kStages = 4;
 constexpr int kTileE = 128;
-constexpr uint32_t kWaitLimit = 1u << 20;  // polls of at most 2 us each
+constexpr uint32_t kWaitLimit = 1u << 22;
 
 struct IdxTcParams {
   IndexerArgs a;

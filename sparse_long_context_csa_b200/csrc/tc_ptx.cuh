@@ -28,26 +28,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// One poll.  If the phase is not complete yet the hardware may suspend the thread until it
-// completes or `suspend_ns` nanoseconds pass, so waiting warps do not flood the shared-memory
-// pipe with polls while copies into shared memory are in flight.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns = 0) {
+// One poll (mbarrier.try_wait: if the phase is not complete the hardware may suspend the
+// thread for a short, implementation-defined time, waking it when the phase completes).
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
-// Bounded wait: returns false after `limit` polls, each suspending for at most `suspend_ns`
-// (so the longest wait is about limit x suspend_ns).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 20),
-                                          uint32_t suspend_ns = 2000) {
+// Bounded wait: returns false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 20)) {
   for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait(bar, parity, suspend_ns)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
 
