@@ -15,10 +15,15 @@
 //
 // Warp roles: 0-3 = producers (entry tiles by 16-byte cp.async into a 4-stage ring; measured
 // on B200, TMA boxes of 128-byte rows streamed at ~1.2 TB/s over the whole GPU, cp.async from
-// four warps per SM at several times that), 4 = MMA issuer and TMEM owner, 5-8 = epilogue
-// (double-buffered TMEM accumulators).  Tiles past the largest visible entry count of the
-// group are skipped (causality).  Grid: (entry splits, query groups).
+// four warps per SM at several times that), 4 = MMA issuer and TMEM owner, 5-12 = epilogue
+// (double-buffered TMEM accumulators; two warps per TMEM lane quadrant, each taking half of
+// the queries of the group).  The epilogue is specialised on the head count so that every
+// 32-column TMEM load turns into whole scores with independent accumulators (measured: a
+// generic per-column loop issued ~6x the instructions and held the kernel at 4% of the
+// tensor pipe).  Tiles past the largest visible entry count of the group are skipped
+// (causality).  Grid: (entry splits, query groups).
 #include <cuda.h>
+#include <cstddef>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -31,7 +36,8 @@ __device__ int g_indexer_tc_error = 0;
 
 namespace {
 
-constexpr int kThreads = 288;  // 4 producer warps, 1 MMA warp, 4 epilogue warps
+constexpr int kThreads = 416;  // 4 producer warps, 1 MMA warp, 8 epilogue warps
+constexpr int kEpilogue = 256;
 constexpr int kProducers = 128;
 constexpr int kStages = 4;
 constexpr int kTileE = 128;
@@ -66,10 +72,64 @@ struct IdxMisc {
   int maxvis;
   int abort_flag;
   int vis[256];
-  float w[256];
+  alignas(16) float w[256 + 32];  // (query, head) weights, read as float4; zero past the group
 };
+static_assert(sizeof(IdxMisc) <= 4096, "misc block exceeds its reservation");
+static_assert(offsetof(IdxMisc, w) % 16 == 0, "weights are read as float4");
 
-__global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcParams P) {
+// Scores of one 32-column chunk of the accumulator (columns c .. c+31, column = q * NI + h)
+// for the entry of this thread: whole queries for NI <= 32; for NI = 64 two chunks make one
+// query (the first leaves its partial sum in `carry`).
+template <int NI>
+__device__ __forceinline__ void score_chunk(const float (&acc)[32], int c, const float* wsm, const int* vis, int nq,
+                                            int w, float* sbase, int64_t P_cap, float& carry) {
+  float wv[32];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 v = *reinterpret_cast<const float4*>(wsm + c + 4 * k);
+    wv[4 * k] = v.x;
+    wv[4 * k + 1] = v.y;
+    wv[4 * k + 2] = v.z;
+    wv[4 * k + 3] = v.w;
+  }
+  if constexpr (NI <= 32) {
+#pragma unroll
+    for (int qq = 0; qq < 32 / NI; ++qq) {
+      float sc = 0.f;
+#pragma unroll
+      for (int h = 0; h < NI; ++h) sc = fmaf(wv[qq * NI + h], fmaxf(acc[qq * NI + h], 0.f), sc);
+      const int q = c / NI + qq;
+      if (q < nq && w < vis[q]) sbase[(int64_t)q * P_cap] = sc;
+    }
+  } else {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int h = 0; h < 32; h += 2) {
+      s0 = fmaf(wv[h], fmaxf(acc[h], 0.f), s0);
+      s1 = fmaf(wv[h + 1], fmaxf(acc[h + 1], 0.f), s1);
+    }
+    if ((c & 63) == 0) {
+      carry = s0 + s1;
+    } else {
+      const int q = c / 64;
+      if (q < nq && w < vis[q]) sbase[(int64_t)q * P_cap] = carry + s0 + s1;
+    }
+  }
+}
+
+// The epilogue of one tile for this thread's chunks [k_lo, k_hi) of 32 columns.
+template <int NI>
+__device__ __forceinline__ void score_tile(uint32_t taddr, int k_lo, int k_hi, const float* wsm, const int* vis,
+                                           int nq, int w, float* sbase, int64_t P_cap) {
+  float carry = 0.f;
+  for (int k = k_lo; k < k_hi; ++k) {
+    float acc[32];
+    tc::tmem_ld_x32(taddr + 32 * k, acc);
+    score_chunk<NI>(acc, 32 * k, wsm, vis, nq, w, sbase, P_cap, carry);
+  }
+}
+
+__global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const IndexerArgs& a = P.a;
   const int cI = a.cI, nI = a.nI, QB = P.QB, Npad = P.Npad;
@@ -98,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&ms->tfull[i], 1);
-      tc::mbar_init(&ms->tempty[i], 128);
+      tc::mbar_init(&ms->tempty[i], kEpilogue);
     }
     ms->maxvis = 0;
     ms->abort_flag = 0;
@@ -121,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
     ms->vis[q] = v;
     atomicMax(&ms->maxvis, v);
   }
-  for (int i = tid; i < QB * nI; i += kThreads) ms->w[i] = (i / nI) < nq ? a.wI[rbase * nI + i] : 0.f;
+  for (int i = tid; i < 256 + 32; i += kThreads) ms->w[i] = (i < QB * nI && (i / nI) < nq) ? a.wI[rbase * nI + i] : 0.f;
   // (query, head) rows -> K-major 128B-swizzled B operand, by cp.async (rows past the group
   // are zero-filled with plain stores)
   {
@@ -211,8 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
       __syncwarp();
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (8 warps)
     const int q4 = warp & 3;
+    const int half = (warp - 5) >> 2;
     const int e = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     // few columns (decode): weights and visibility live in registers for the whole CTA
@@ -224,43 +285,43 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcPara
       qcol[j] = j >> lg_nI;
       wsm[j] = (small && qcol[j] < nq) ? ms->w[j] : 0.f;
     }
+    // 32-column chunks of this half: whole queries (two chunks per query when nI = 64)
+    const int nchk = (Npad + 31) / 32;
+    const int cpq = nI > 32 ? 2 : 1;
+    const int units = (nchk + cpq - 1) / cpq;
+    const int u_mid = (units + 1) / 2;
+    const int k_lo = half == 0 ? 0 : u_mid * cpq;
+    const int k_hi = half == 0 ? min(nchk, u_mid * cpq) : nchk;
     for (int i = 0; i < ntiles; ++i) {
       const int tb = i & 1;
-      if (!tc::named_bar_and(1, 128, tc::mbar_wait(&ms->tfull[tb], (i >> 1) & 1, kWaitLimit))) {
-        if (e == 0) atomicExch(&g_indexer_tc_error, 5);
+      if (!tc::named_bar_and(1, kEpilogue, tc::mbar_wait(&ms->tfull[tb], (i >> 1) & 1, kWaitLimit))) {
+        if (tid == 160) atomicExch(&g_indexer_tc_error, 5);
         break;
       }
       tc::tc_fence_after();
       const int w = (t_lo + i) * kTileE + e;
       if (small) {
-        float acc[16];
-        tc::tmem_ld_x16(tmem + tb * Npad + lane_off, acc);
-        for (int q = 0; q < nq; ++q) {
-          float sc = 0.f;
+        if (half == 0) {
+          float acc[16];
+          tc::tmem_ld_x16(tmem + tb * Npad + lane_off, acc);
+          for (int q = 0; q < nq; ++q) {
+            float sc = 0.f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) sc = fmaf(qcol[j] == q ? wsm[j] : 0.f, fmaxf(acc[j], 0.f), sc);
-          if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
-        }
-        tc::tc_fence_before();
-        tc::mbar_arrive(&ms->tempty[tb]);
-        continue;
-      }
-      // 16 accumulator columns at a time, column = q * nI + h (nI is a power of two)
-      float sc = 0.f;
-      for (int c0 = 0; c0 < Npad; c0 += 16) {
-        float acc[16];
-        tc::tmem_ld_x16(tmem + tb * Npad + c0 + lane_off, acc);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int col = c0 + j;
-          const int q = col >> lg_nI, h = col & (nI - 1);
-          if (q < nq) {
-            sc = fmaf(ms->w[col], fmaxf(acc[j], 0.f), sc);
-            if (h == nI - 1) {
-              if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
-              sc = 0.f;
-            }
+            for (int j = 0; j < 16; ++j) sc = fmaf(qcol[j] == q ? wsm[j] : 0.f, fmaxf(acc[j], 0.f), sc);
+            if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
           }
+        }
+      } else {
+        float* sbase = a.scores + (rbase - P.row0) * a.P_cap + w;
+        const uint32_t taddr = tmem + tb * Npad + lane_off;
+        switch (nI) {
+          case 1: score_tile<1>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 2: score_tile<2>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 4: score_tile<4>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 8: score_tile<8>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 16: score_tile<16>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 32: score_tile<32>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          default: score_tile<64>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
         }
       }
       tc::tc_fence_before();
