@@ -211,10 +211,24 @@ __global__ void __launch_bounds__(NT) topk_kernel(IndexerArgs a, int64_t row0) {
   const bool cached = vis <= kTopkSmemKeys;
   for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
   __syncthreads();
-  for (int i = tid; i < vis; i += NT) {
-    const uint32_t k = order_key(sc[i]);
-    if (cached) keys[i] = k;
-    atomicAdd(&hist[k >> 20], 1u);
+  // Eight score loads per thread are issued before any is used, so a long row costs a few
+  // memory round trips instead of one per key.
+  for (int base = tid; base < vis; base += NT * 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = base + u * NT;
+      v[u] = j < vis ? sc[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = base + u * NT;
+      if (j < vis) {
+        const uint32_t k = order_key(v[u]);
+        if (cached) keys[j] = k;
+        atomicAdd(&hist[k >> 20], 1u);
+      }
+    }
   }
   __syncthreads();
   find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
