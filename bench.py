@@ -108,7 +108,12 @@ def roofline_of(name, flops, nbytes, ms, peaks, peak_src):
 # kernel, from one ncu capture of that kernel on that workload, keyed by the SHA-256 of the
 # kernel's source file when it was captured: once the kernel changes, traffic reads null
 # until it is captured again.  Values: (source file, sha256, bytes per launch).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
+    # window 128): dram__bytes_read.sum 564.3 MB + dram__bytes_write.sum 494.1 MB.
+    ("csa_prefill_bf16", "attention"): (
+        "attn_tc.cu", "12f841fcc4fc42d7f4fbc29246dfb904d709de1570fe2a5bdcecf12ee7c1faf5", 1058375936),
+}
 PART_SOURCE = {"attention": "attn_tc.cu", "indexer_scores": "indexer_tc.cu", "topk": "indexer.cu",
                "compress": "compress.cu"}
 

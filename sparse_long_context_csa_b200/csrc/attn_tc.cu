@@ -61,7 +61,7 @@ constexpr int kThreads = 320;  // 10 warps
 constexpr int kMaxChunks = 9;  // D <= 576
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
-constexpr uint32_t kWaitLimit = 1u << 20;  // polls of at most 2 us each: a stuck wait ends in ~2 s
+constexpr uint32_t kWaitLimit = 1u << 20;  // mbarrier polls before a wait gives up
 
 struct TcParams {
   AttnArgs a;
