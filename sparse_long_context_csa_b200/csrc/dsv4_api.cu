@@ -24,6 +24,13 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
 
+// Keys a query attends at most: the window plus the selected (top-k) or all pool entries.
+// Only the sizes enter, so the workspace size and the launch agree on the key split.
+int64_t attn_keys_estimate(const dsv4_params* p) {
+  const int64_t pool = p->topk > 0 ? (p->topk < p->P_cap ? p->topk : p->P_cap) : p->P_cap;
+  return (int64_t)(p->n_win > 0 ? p->n_win : 0) + (pool > 0 ? pool : 0);
+}
+
 dsv4_status check_common(const dsv4_params* p) {
   if (!p) return DSV4_ERR_ARG;
   if (p->dtype != DSV4_F32 && p->dtype != DSV4_BF16) return DSV4_ERR_DTYPE;
@@ -127,10 +134,10 @@ dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, co
   if (rows == 0) return DSV4_OK;
   if (attn_tc_supported(a, p->dtype)) {
     // few queries: split each query's keys over several CTAs when a workspace is given
-    const size_t need = attn_split_bytes(rows, p->dv);
+    const size_t need = attn_split_bytes(rows, attn_keys_estimate(p), p->dv);
     if (need > 0 && workspace && ws_bytes >= need) {
       a.part = static_cast<float*>(workspace);
-      a.nsplit = attn_splits(rows);
+      a.nsplit = attn_splits(rows, attn_keys_estimate(p));
     }
     return from_cuda(launch_attn_tc(a, as_stream(stream)));
   }
@@ -185,7 +192,7 @@ dsv4_status dsv4_device_check(void* stream) {
 size_t dsv4_workspace_bytes(const dsv4_params* p) {
   if (!p || check_common(p) != DSV4_OK) return 0;
   const size_t layer = align_up(layer_idx_bytes(p)) + align_up(scores_bytes(p));
-  const size_t attn = align_up(attn_split_bytes((int64_t)p->B * p->Sq, p->dv));
+  const size_t attn = align_up(attn_split_bytes((int64_t)p->B * p->Sq, attn_keys_estimate(p), p->dv));
   return layer > attn ? layer : attn;  // the attention partials reuse the indexer's scores space
 }
 

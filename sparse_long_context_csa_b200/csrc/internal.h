@@ -65,10 +65,11 @@ struct AttnArgs {
   float* part;  // split-over-keys partials (workspace) or nullptr
   int nsplit;   // key splits per query (1 = no split)
 };
-// Key splits per query used by the tensor-core attention for B*Sq queries (a pure function
-// of the sizes, so that the workspace size is one too), and the workspace it needs.
-int attn_splits(int64_t rows);
-size_t attn_split_bytes(int64_t rows, int dv);
+// Key splits per query used by the tensor-core attention for B*Sq queries attending about
+// keys_per_query keys each (a pure function of the sizes, so that the workspace size is one
+// too), and the workspace it needs.
+int attn_splits(int64_t rows, int64_t keys_per_query);
+size_t attn_split_bytes(int64_t rows, int64_t keys_per_query, int dv);
 cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 // Tensor-core (tcgen05) path; returns cudaErrorNotSupported when the shape is not covered.
 bool attn_tc_supported(const AttnArgs& a, int dtype);

@@ -145,7 +145,8 @@ def test_workspace_is_a_pure_function_of_params(abi):
     assert sizes["hca_prefill_bf16"] == 0                      # no indexer
     assert sizes["csa_prefill_bf16"] == 8192 * 512 * 4 + 8192 * 2048 * 4
     # decode keeps no layer idx; its attention partials (5 key splits x 64 queries) dominate
-    assert sizes["csa_decode_bf16"] == max(64 * 32768 * 4, 64 * 5 * 64 * (512 + 2) * 4)
+    # 64 queries of 128 window + 2048 selected keys: two key splits per query
+    assert sizes["csa_decode_bf16"] == max(64 * 32768 * 4, 64 * 2 * 64 * (512 + 2) * 4)
     assert sizes["dsa_prefill_bf16"] == 32768 * 2048 * 4 + (256 << 20)
     assert abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"])) == \
         abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"]))

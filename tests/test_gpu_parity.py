@@ -215,12 +215,13 @@ def test_sparse_attention_kernel(lib, name, gains, use_idx):
         assert_max_abs(g[b, s], ref[b, s], ATTN_TOL[w.dtype], f"{name} row {(b, s)}")
 
 
-@pytest.mark.parametrize("B,with_ws", [(3, True), (3, False), (40, True)])
-def test_decode_attention_key_splits(lib, B, with_ws):
+@pytest.mark.parametrize("B,with_ws,S", [(3, True, 20000), (3, False, 20000), (40, True, 20000), (3, True, 600)])
+def test_decode_attention_key_splits(lib, B, with_ws, S):
     """Few queries: the keys of each query are split over CTAs and merged (or not, without a
-    workspace); 3 sequences give 16 splits, several of them empty."""
+    workspace).  The split count comes from the sizes (window + top-k keys); with S=600 the
+    caches hold at most 150 entries, so most of the 9 splits of a query are empty."""
     abi, harness = lib
-    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, S=20000, P_cap=5000, topk=1024, qindex_spread=500)
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, S=S, P_cap=5000, topk=1024, qindex_spread=500)
     c = _cache(w, {"q": 256.0})
     x = _query_inputs(w, {"q": 256.0})
     idx = synth.strided_selection(w, x["q_index"])
