@@ -105,30 +105,42 @@ def roofline_of(name, flops, nbytes, ms, peaks, peak_src):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a part's main
-# kernel, from one ncu capture of that kernel on that workload, keyed by the SHA-256 of the
-# kernel's source file when it was captured: once the kernel changes, traffic reads null
-# until it is captured again.  Values: (source file, sha256, bytes per launch).
+# kernel, from one ncu capture of that kernel on that workload.  Each record carries the
+# SHA-256 of the source that makes up the kernel at capture time (its file up to the end of
+# the kernel definition, and the headers it includes): once any of it changes, traffic reads
+# null until the kernel is captured again.  Values: (source segments, sha256, bytes per launch).
+_ATTN_SOURCE = (("attn_tc.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("common.cuh", None),
+                ("internal.h", None))
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
     # window 128): dram__bytes_read.sum 564.3 MB + dram__bytes_write.sum 494.1 MB.
-    ("csa_prefill_bf16", "attention"): (
-        "attn_tc.cu", "12f841fcc4fc42d7f4fbc29246dfb904d709de1570fe2a5bdcecf12ee7c1faf5", 1058375936),
+    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "75de456acf974ede70a65f460d38300dd361f15d3c325367bd5c59240c83f9ee", 1058375936),
 }
-PART_SOURCE = {"attention": "attn_tc.cu", "indexer_scores": "indexer_tc.cu", "topk": "indexer.cu",
-               "compress": "compress.cu"}
+
+
+def kernel_source_sha(segments) -> str | None:
+    """SHA-256 over the kernel's source segments (a file up to an end marker, or whole)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name, end in segments:
+        try:
+            text = open(os.path.join(ROOT, "sparse_long_context_csa_b200", "csrc", name)).read()
+        except OSError:
+            return None
+        if end is not None:
+            k = text.find(end)
+            if k < 0:
+                return None
+            text = text[:k]
+        h.update(text.encode())
+    return h.hexdigest()
 
 
 def ncu_traffic(workload: str, part: str):
     rec = NCU_TRAFFIC.get((workload, part))
     if rec is None:
         return None
-    import hashlib
-    path = os.path.join(ROOT, "sparse_long_context_csa_b200", "csrc", rec[0])
-    try:
-        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()
-    except OSError:
-        return None
-    return rec[2] if sha == rec[1] else None
+    return rec[2] if kernel_source_sha(rec[0]) == rec[1] else None
 
 
 class ClockSampler:
