@@ -335,3 +335,57 @@ def hca_layer(q, kv, z, bias, sink, pos, *, m, n_win, scale, dv, R, theta, rotat
                                scale=scale, dv=dv, R=R, theta=theta, rope_q=True,
                                rotate_out=rotate_out, rows=rows)
     return {"pool": pool, "kv_rot": kv_rot, "out": out}
+
+
+# --------------------------------------------------------------------------
+# Decode cache  [V4] "Cache layers": the CSA / HCA cache keeps the sliding window of
+# K=V rows and the compressor's buffer of the tokens of the open window(s) (for CSA the
+# previous block too: the overlap state); an entry is emitted every m tokens.  The
+# indexer keys keep a buffer and a pool of their own.
+# --------------------------------------------------------------------------
+def new_decode_cache(c, *, m, overlap, P_cap, win_ring=0):
+    """Empty cache of one stream of one sequence: a buffer of the last Lw = 2m (overlap)
+    or m raw token rows with their logits and positions, an optional window ring and the
+    pool."""
+    lw = 2 * m if overlap else m
+    return {"raw": np.zeros((lw, c)), "z": np.zeros((lw, c)), "pos": np.zeros(lw, dtype=np.int64),
+            "win": np.zeros((win_ring, c)) if win_ring else None, "pool": np.zeros((P_cap, c))}
+
+
+def decode_append(cache, x_t, z_t, pos_t, t, *, m, overlap, bias, apply_rope, R=0, theta=160000.0):
+    """Append token t (cache index) of one sequence: row x_t [c] (not rotated), logits z_t
+    [c] or None, position pos_t.  Tokens must arrive in order t = 0, 1, 2, ...
+
+    The buffer holds token j in slot j % Lw; the window ring holds token j rotated at its
+    position in slot j % win_ring.  When t closes a block ((t+1) % m == 0), entry
+    w = (t+1)/m - 1 is pooled from the buffered tokens of its window (readings R1-R3: the
+    softmax over z + the per-slot bias, rotated at the position of the first token of its
+    own block) and written to the pool if w < P_cap.
+    """
+    lw = cache["raw"].shape[0]
+    c = cache["raw"].shape[1]
+    cache["raw"][t % lw] = _f64(x_t)
+    cache["z"][t % lw] = 0.0 if z_t is None else _f64(z_t)
+    cache["pos"][t % lw] = pos_t
+    if cache["win"] is not None:
+        row = rope_rotate(_f64(x_t), pos_t, R, theta) if apply_rope else _f64(x_t)
+        cache["win"][t % cache["win"].shape[0]] = row
+    if (t + 1) % m != 0:
+        return
+    w = (t + 1) // m - 1
+    if w >= cache["pool"].shape[0]:
+        return
+    lo = (w - 1) * m if overlap else w * m
+    tokens = [j for j in range(max(lo, 0), t + 1)]
+    logit = np.zeros((len(tokens), c))
+    for k, j in enumerate(tokens):
+        logit[k] = cache["z"][j % lw]
+        if bias is not None:
+            logit[k] = logit[k] + _f64(bias)[j - lo]
+    mx = logit.max(axis=0)
+    e = np.exp(logit - mx)
+    alpha = e / e.sum(axis=0)
+    entry = sum(alpha[k] * cache["raw"][j % lw] for k, j in enumerate(tokens))
+    if apply_rope:
+        entry = rope_rotate(entry, cache["pos"][(w * m) % lw], R, theta)
+    cache["pool"][w] = entry

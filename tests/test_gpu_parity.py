@@ -314,3 +314,31 @@ def test_layer_is_deterministic(lib):
     torch.cuda.synchronize()
     assert torch.equal(o1["idx"], o2["idx"])
     assert torch.equal(o1["out"].view(torch.int16), o2["out"].view(torch.int16))
+
+
+@pytest.mark.parametrize("name,gains", [("tiny_csa_f32", None), ("csa_prefill_bf16", None),
+                                        ("csa_prefill_bf16", {"q": 256.0})])
+def test_sliding_window_only_attention(lib, name, gains):
+    """`sliding_attention` layers ("DeepSeek-V4", layer types): the window branch alone — no
+    pool, no index lists (pool NULL, P_cap 0) — over rows already rotated at their positions."""
+    abi, harness = lib
+    w0 = synth.WORKLOADS[name]
+    w = w0.replace(S=min(w0.S, 1024), Sq=min(w0.S, 1024), P_cap=0, topk=0, nI=0)
+    specs = synth.tensor_specs(w, gains)
+    q = synth.reshape(w, "q", specs["q"].full())
+    kv = synth.reshape(w, "kv", specs["kv"].full())
+    sink = specs["sink"].full()
+    qi, qp = synth.positions(w)
+    params = harness.params_for(w)
+    d = harness.to_device(w, {"q": q, "kv": kv, "sink": sink, "qpos": qp, "q_index": qi})
+    out = torch.empty((w.B, w.Sq, w.H, w.dv), dtype=harness.torch_dtype(w), device="cuda")
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(params), 256), dtype=torch.uint8, device="cuda")
+    abi.dsv4_sparse_mqa_attn(params, d["q"], d["kv"], None, None, d["sink"], d["qpos"], d["q_index"], out, ws)
+    abi.dsv4_device_check()
+    rows = [(0, s) for s in sample_rows(w.Sq, 128, 16)]
+    ref = O.sparse_mqa_attention(q, kv, np.zeros((w.B, 0, w.D)), None, sink, qp, qi, n_win=w.n_win, m=w.m,
+                                 scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rope_q=True,
+                                 rotate_out=w.rotate_out, P_cap=0, rows=rows)
+    g = _np(out)
+    for b, s in rows:
+        assert_max_abs(g[b, s], ref[b, s], ATTN_TOL[w.dtype], f"{name} window-only row {(b, s)}")

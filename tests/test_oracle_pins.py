@@ -419,3 +419,30 @@ def test_dsa_token_level_includes_self():
     out = O.sparse_mqa_attention(q, np.zeros((1, S, D)), pool, None, sink, qi, qi, n_win=0, m=1,
                                  scale=1.0, dv=D, R=2, theta=10.0, rope_q=False, rotate_out=False)
     np.testing.assert_allclose(out[0, 0], np.tile(pool[0, 0], (H, 1)), atol=1e-14)
+
+
+# ---------------------------------------------------------------- decode cache
+@pytest.mark.parametrize("m,overlap", [(4, True), (8, False), (1, False)])
+def test_decode_append_matches_prefill_compression(m, overlap):
+    """Appending tokens one at a time through the decode cache ("Cache layers": window ring
+    and compressor buffer with its overlap state) gives the pool that compressing the
+    whole prefix at once gives, and a window ring holding the last rows rotated at their
+    positions; entries past the pool capacity are not written, and a partial last block
+    is not an entry."""
+    rng = np.random.default_rng(11)
+    S, c, R, ring = 37, 16, 8, 16
+    lw = 2 * m if overlap else m
+    x = rng.standard_normal((1, S, c))
+    z = rng.standard_normal((1, S, c))
+    bias = 0.3 * rng.standard_normal((lw, c))
+    pos = (np.arange(S) * 3 + 1000)[None]            # positions are not the cache indices
+    batch = O.compress(x, z, bias, pos, m=m, overlap=overlap, apply_rope=True, R=R, theta=10000.0)
+    P_cap = S // m - 1                                # the last complete entry does not fit
+    cache = O.new_decode_cache(c, m=m, overlap=overlap, P_cap=P_cap, win_ring=ring)
+    for t in range(S):
+        O.decode_append(cache, x[0, t], z[0, t], pos[0, t], t, m=m, overlap=overlap, bias=bias,
+                        apply_rope=True, R=R, theta=10000.0)
+    np.testing.assert_allclose(cache["pool"], batch[0, :P_cap], rtol=0, atol=1e-12)
+    rot = O.rope_rotate(x, pos, R, 10000.0)
+    for j in range(S - ring, S):
+        np.testing.assert_allclose(cache["win"][j % ring], rot[0, j], rtol=0, atol=1e-12)
