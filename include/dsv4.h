@@ -105,6 +105,40 @@ dsv4_status dsv4_compress_kv(const dsv4_params* params, int32_t c, const void* x
                              void* pool, void* x_rot, void* stream);
 
 /*
+ * Decode-cache append ([V4] "Cache layers": the CSA / HCA cache keeps the sliding window of
+ * K=V rows and the compressor's buffer of the tokens of the open window(s) -- for CSA the
+ * previous block too, its overlap state; an entry is emitted every m tokens; the indexer
+ * keys keep a buffer and a pool of their own).
+ *
+ * Appends one token to each of B sequences.  Sequence b's new token has cache index t[b]
+ * (t[b] < 0: the sequence is skipped); the tokens of a sequence must be appended in order
+ * t = 0, 1, 2, ...  When the token closes a block ((t+1) % m == 0), entry w = (t+1)/m - 1 is
+ * pooled from the buffer and written if w < P_cap: the same pooling and RoPE as
+ * dsv4_compress_kv, with the same arithmetic, so the entry has the same bits as the one
+ * dsv4_compress_kv writes for the same token rows.  Lw = 2m with overlap, else m.
+ *
+ *   c          channels per row (D for the K=V stream, cI for the indexer keys); even
+ *   x          [B,c] T             the new tokens' rows (not rotated)
+ *   z          [B,c] T or NULL     their compressor logits (NULL = 0)
+ *   bias       [Lw,c] f32 or NULL  per-slot bias
+ *   pos        [B] int64           the new tokens' positions
+ *   t          [B] int32           the new tokens' cache indices
+ *   buf_x      [B,Lw,c] T          in/out: raw rows of the last Lw tokens (token j in slot j % Lw)
+ *   buf_z      [B,Lw,c] T or NULL  in/out: their logits (required when z is given)
+ *   buf_pos    [B,Lw] int64        in/out: their positions
+ *   apply_rope rotate the window rows and the new entries (trailing R channels, rope_theta)
+ *   win        [B,win_ring,c] T or NULL  in/out: window ring; token j, rotated at its
+ *                                  position when apply_rope, in slot j % win_ring
+ *   pool       [B,P_cap,c] T       in/out: the pool
+ * Uses B, m, overlap, win_ring, P_cap, R, rope_theta and dtype from params.  Validates on the
+ * host (DSV4_ERR_ARG / _SHAPE / _ALIGN / _DTYPE) before any launch; allocates nothing.
+ */
+dsv4_status dsv4_decode_append(const dsv4_params* params, int32_t c, const void* x, const void* z,
+                               const float* bias, const int64_t* pos, const int32_t* t, void* buf_x,
+                               void* buf_z, int64_t* buf_pos, int32_t apply_rope, void* win, void* pool,
+                               void* stream);
+
+/*
  * Lightning Indexer + top-k ([V4] CSA item, eqs. 13-17 and index_topk (eq. 17);
  * [V32] DSA items 1-2).  For each query (b,s) at cache index t = q_index[b,s] and
  * every visible entry w < vis = min((t+1)/m, P_cap):

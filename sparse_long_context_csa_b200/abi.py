@@ -21,7 +21,7 @@ STATUS = {0: "DSV4_OK", 1: "DSV4_ERR_ARG", 2: "DSV4_ERR_SHAPE", 3: "DSV4_ERR_ALI
 EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
             "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check", "dsv4_indexer_scores",
-            "dsv4_topk_select")
+            "dsv4_topk_select", "dsv4_decode_append")
 
 
 class Dsv4Error(RuntimeError):
@@ -60,6 +60,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_indexer_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.dsv4_indexer_scores.argtypes = [P, vp, vp, vp, vp, vp, vp]
     lib.dsv4_topk_select.argtypes = [P, vp, vp, vp, vp]
+    lib.dsv4_decode_append.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.dsv4_sparse_mqa_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_csa_layer.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.dsv4_hca_layer.argtypes = [P] + [vp] * 10 + [sz, vp]
@@ -72,7 +73,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_device_check.argtypes = [vp]
     lib.dsv4_device_check.restype = ctypes.c_int
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
-               "dsv4_hca_layer", "dsv4_indexer_topk_noalloc", "dsv4_indexer_scores", "dsv4_topk_select"):
+               "dsv4_hca_layer", "dsv4_indexer_topk_noalloc", "dsv4_indexer_scores", "dsv4_topk_select",
+               "dsv4_decode_append"):
         getattr(lib, fn).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -141,6 +143,13 @@ def dsv4_topk_select(params, scores, q_index, idx, stream=None):
     """Per-query top-k over given score rows: idx[B,Sq,topk] ascending entries, then -1."""
     _check("dsv4_topk_select", load().dsv4_topk_select(
         ctypes.byref(params), _ptr(scores), _ptr(q_index), _ptr(idx), _stream(stream)))
+
+
+def dsv4_decode_append(params, c, x, z, bias, pos, t, buf_x, buf_z, buf_pos, apply_rope, win, pool, stream=None):
+    """Append one token per sequence to the decode cache (buffer, window ring, pool)."""
+    _check("dsv4_decode_append", load().dsv4_decode_append(
+        ctypes.byref(params), c, _ptr(x), _ptr(z), _ptr(bias), _ptr(pos), _ptr(t), _ptr(buf_x), _ptr(buf_z),
+        _ptr(buf_pos), apply_rope, _ptr(win), _ptr(pool), _stream(stream)))
 
 
 def dsv4_sparse_mqa_attn(params, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace=None,

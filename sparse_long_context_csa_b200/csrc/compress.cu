@@ -17,6 +17,60 @@
 
 namespace dsv4 {
 
+// Softmax-gated pooling of channel pair (d, d+1) over tokens j = j0 .. hi-1 of one entry
+// window starting at token lo (slot j - lo of the bias); row_of(j) is the row holding token
+// j.  An online (running max) softmax in fp32.  Shared by the prefill compressor and the
+// decode-cache append, so that both write the same bits for the same rows.
+template <typename T, typename RowOf>
+__device__ __forceinline__ float2 pool_pair(const T* __restrict__ x, const T* __restrict__ z,
+                                            const float* __restrict__ bias, int lo, int j0, int hi, int c, int d,
+                                            RowOf row_of) {
+  float mx0 = -INFINITY, mx1 = -INFINITY, s0 = 0.f, s1 = 0.f, acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 4
+  for (int j = j0; j < hi; ++j) {
+    const int64_t r = row_of(j);
+    const float2 xv = load2<T>(x + r * c + d);
+    float l0 = 0.f, l1 = 0.f;
+    if (z) {
+      const float2 zv = load2<T>(z + r * c + d);
+      l0 = zv.x;
+      l1 = zv.y;
+    }
+    if (bias) {
+      const float2 bv = *reinterpret_cast<const float2*>(bias + (int64_t)(j - lo) * c + d);
+      l0 += bv.x;
+      l1 += bv.y;
+    }
+    if (l0 > mx0) {
+      const float q = expf(mx0 - l0);
+      s0 *= q;
+      acc0 *= q;
+      mx0 = l0;
+    }
+    if (l1 > mx1) {
+      const float q = expf(mx1 - l1);
+      s1 *= q;
+      acc1 *= q;
+      mx1 = l1;
+    }
+    const float e0 = expf(l0 - mx0), e1 = expf(l1 - mx1);
+    s0 += e0;
+    s1 += e1;
+    acc0 = fmaf(e0, xv.x, acc0);
+    acc1 = fmaf(e1, xv.y, acc1);
+  }
+  return make_float2(acc0 / s0, acc1 / s1);
+}
+
+// RoPE of channel pair (d, d+1) when it lies in the trailing R channels.
+__device__ __forceinline__ float2 rope_pair(float2 v, int64_t pos, int d, int c, int R, float theta) {
+  const int rope_lo = c - R;
+  if (d < rope_lo) return v;
+  float cs, sn;
+  rope_cos_sin(pos, (d - rope_lo) / 2, R, theta, &cs, &sn);
+  return make_float2(v.x * cs - v.y * sn, v.x * sn + v.y * cs);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
   const int w = blockIdx.x;
@@ -28,7 +82,6 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
   const T* __restrict__ x = static_cast<const T*>(a.x) + (int64_t)b * S * c;
   const T* __restrict__ z = a.z ? static_cast<const T*>(a.z) + (int64_t)b * S * c : nullptr;
   const int64_t* pos = a.pos ? a.pos + (int64_t)b * S : nullptr;
-  const int rope_lo = c - a.R;
 
   if (w < P) {
     const int lo = a.overlap ? (w - 1) * m : w * m;
@@ -37,49 +90,9 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
     T* __restrict__ pool = static_cast<T*>(a.pool) + ((int64_t)b * a.P_cap + w) * c;
     for (int pr = threadIdx.x; pr < c / 2; pr += blockDim.x) {
       const int d = 2 * pr;
-      float mx0 = -INFINITY, mx1 = -INFINITY, s0 = 0.f, s1 = 0.f, acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 4
-      for (int j = j0; j < hi; ++j) {
-        const float2 xv = load2<T>(x + (int64_t)j * c + d);
-        float l0 = 0.f, l1 = 0.f;
-        if (z) {
-          const float2 zv = load2<T>(z + (int64_t)j * c + d);
-          l0 = zv.x;
-          l1 = zv.y;
-        }
-        if (a.bias) {
-          const float2 bv = *reinterpret_cast<const float2*>(a.bias + (int64_t)(j - lo) * c + d);
-          l0 += bv.x;
-          l1 += bv.y;
-        }
-        if (l0 > mx0) {
-          const float r = expf(mx0 - l0);
-          s0 *= r;
-          acc0 *= r;
-          mx0 = l0;
-        }
-        if (l1 > mx1) {
-          const float r = expf(mx1 - l1);
-          s1 *= r;
-          acc1 *= r;
-          mx1 = l1;
-        }
-        const float e0 = expf(l0 - mx0), e1 = expf(l1 - mx1);
-        s0 += e0;
-        s1 += e1;
-        acc0 = fmaf(e0, xv.x, acc0);
-        acc1 = fmaf(e1, xv.y, acc1);
-      }
-      float v0 = acc0 / s0, v1 = acc1 / s1;
-      if (a.apply_rope && d >= rope_lo) {
-        float cs, sn;
-        rope_cos_sin(pos[(int64_t)w * m], (d - rope_lo) / 2, a.R, a.theta, &cs, &sn);
-        const float r0 = v0 * cs - v1 * sn;
-        const float r1 = v0 * sn + v1 * cs;
-        v0 = r0;
-        v1 = r1;
-      }
-      store2<T>(pool + d, v0, v1);
+      float2 v = pool_pair<T>(x, z, a.bias, lo, j0, hi, c, d, [](int j) { return (int64_t)j; });
+      if (a.apply_rope) v = rope_pair(v, pos[(int64_t)w * m], d, c, a.R, a.theta);
+      store2<T>(pool + d, v.x, v.y);
     }
   }
 
@@ -90,14 +103,7 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
     for (int it = threadIdx.x; it < (t_hi - w * m) * npairs; it += blockDim.x) {
       const int j = w * m + it / npairs;
       const int d = 2 * (it % npairs);
-      float2 v = load2<T>(x + (int64_t)j * c + d);
-      if (d >= rope_lo) {
-        float cs, sn;
-        rope_cos_sin(pos[j], (d - rope_lo) / 2, a.R, a.theta, &cs, &sn);
-        const float r0 = v.x * cs - v.y * sn;
-        const float r1 = v.x * sn + v.y * cs;
-        v = make_float2(r0, r1);
-      }
+      const float2 v = rope_pair(load2<T>(x + (int64_t)j * c + d), pos[j], d, c, a.R, a.theta);
       store2<T>(xr + (int64_t)j * c + d, v.x, v.y);
     }
   }
@@ -113,6 +119,64 @@ cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st) {
     compress_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(a);
   else
     compress_kernel<float><<<grid, threads, 0, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// Decode-cache append: one CTA per sequence, thread per channel pair.  The new token goes to
+// buffer slot t % Lw (raw row, logits, position) and, rotated, to window-ring slot
+// t % win_ring; when it closes a block, the entry of that block is pooled from the buffer.
+// A thread reads back only the channels it wrote itself; the buffered positions, written by
+// thread 0, are read after a barrier.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_append_kernel(DecodeAppendArgs a) {
+  const int b = blockIdx.x;
+  const int t = a.t[b];
+  if (t < 0) return;
+  const int c = a.c, m = a.m;
+  const int lw = a.overlap ? 2 * m : m;
+  const int64_t pos = a.pos[b];
+  const T* __restrict__ xn = static_cast<const T*>(a.x) + (int64_t)b * c;
+  const T* __restrict__ zn = a.z ? static_cast<const T*>(a.z) + (int64_t)b * c : nullptr;
+  T* __restrict__ bx = static_cast<T*>(a.buf_x) + (int64_t)b * lw * c;
+  T* __restrict__ bz = a.buf_z ? static_cast<T*>(a.buf_z) + (int64_t)b * lw * c : nullptr;
+  const int slot = t % lw;
+  for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
+    const float2 xv = load2<T>(xn + d);
+    store2<T>(bx + (int64_t)slot * c + d, xv.x, xv.y);
+    if (bz) {
+      const float2 zv = zn ? load2<T>(zn + d) : make_float2(0.f, 0.f);
+      store2<T>(bz + (int64_t)slot * c + d, zv.x, zv.y);
+    }
+    if (a.win) {
+      const float2 v = a.apply_rope ? rope_pair(xv, pos, d, c, a.R, a.theta) : xv;
+      store2<T>(static_cast<T*>(a.win) + ((int64_t)b * a.win_ring + t % a.win_ring) * c + d, v.x, v.y);
+    }
+  }
+  if (threadIdx.x == 0) a.buf_pos[(int64_t)b * lw + slot] = pos;
+  __syncthreads();
+  if ((t + 1) % m != 0) return;
+  const int w = (t + 1) / m - 1;
+  if (w >= a.P_cap) return;
+  const int lo = a.overlap ? (w - 1) * m : w * m;
+  const int j0 = lo < 0 ? 0 : lo;
+  const int64_t epos = a.buf_pos[(int64_t)b * lw + (w * m) % lw];
+  T* __restrict__ pool = static_cast<T*>(a.pool) + ((int64_t)b * a.P_cap + w) * c;
+  for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
+    float2 v = pool_pair<T>(bx, bz, a.bias, lo, j0, t + 1, c, d, [lw](int j) { return (int64_t)(j % lw); });
+    if (a.apply_rope) v = rope_pair(v, epos, d, c, a.R, a.theta);
+    store2<T>(pool + d, v.x, v.y);
+  }
+}
+
+cudaError_t launch_decode_append(const DecodeAppendArgs& a, int dtype, cudaStream_t st) {
+  if (a.B == 0) return cudaSuccess;
+  int threads = ((a.c / 2 + 31) / 32) * 32;
+  threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
+  if (dtype == DSV4_BF16)
+    decode_append_kernel<__nv_bfloat16><<<a.B, threads, 0, st>>>(a);
+  else
+    decode_append_kernel<float><<<a.B, threads, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }

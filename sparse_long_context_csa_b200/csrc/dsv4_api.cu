@@ -203,6 +203,28 @@ dsv4_status dsv4_compress_kv(const dsv4_params* p, int32_t c, const void* x, con
   return run_compress(p, c, x, z, bias, pos, apply_rope, pool, x_rot, stream);
 }
 
+dsv4_status dsv4_decode_append(const dsv4_params* p, int32_t c, const void* x, const void* z, const float* bias,
+                               const int64_t* pos, const int32_t* t, void* buf_x, void* buf_z, int64_t* buf_pos,
+                               int32_t apply_rope, void* win, void* pool, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if (c < 2 || (c & 1)) return DSV4_ERR_SHAPE;
+  if (!x || !pos || !t || !buf_x || !buf_pos || !pool) return DSV4_ERR_ARG;
+  if (z && !buf_z) return DSV4_ERR_ARG;  // logits can only be pooled from the buffer
+  if (win && p->win_ring < 1) return DSV4_ERR_SHAPE;
+  if (apply_rope != 0 && apply_rope != 1) return DSV4_ERR_ARG;
+  if (apply_rope && (p->R < 0 || (p->R & 1) || p->R > c || !(p->rope_theta > 0.f))) return DSV4_ERR_SHAPE;
+  const void* ptrs[] = {x, z, bias, pos, t, buf_x, buf_z, buf_pos, win, pool};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return DSV4_ERR_ALIGN;
+  DecodeAppendArgs a{};
+  a.B = p->B; a.c = c; a.m = p->m; a.overlap = p->overlap; a.win_ring = p->win_ring; a.P_cap = p->P_cap;
+  a.R = apply_rope ? p->R : 0; a.apply_rope = apply_rope; a.theta = p->rope_theta;
+  a.x = x; a.z = z; a.bias = bias; a.pos = pos; a.t = t; a.buf_x = buf_x; a.buf_z = buf_z; a.buf_pos = buf_pos;
+  a.win = win; a.pool = pool;
+  return from_cuda(launch_decode_append(a, p->dtype, as_stream(stream)));
+}
+
 dsv4_status dsv4_indexer_topk(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
                               const int32_t* q_index, int32_t* idx, void* workspace, size_t ws_bytes,
                               void* stream) {

@@ -25,6 +25,22 @@ struct CompressArgs {
 };
 cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st);
 
+struct DecodeAppendArgs {
+  int B, c, m, overlap, win_ring, P_cap, R, apply_rope;
+  float theta;
+  const void* x;
+  const void* z;
+  const float* bias;
+  const int64_t* pos;
+  const int32_t* t;
+  void* buf_x;
+  void* buf_z;
+  int64_t* buf_pos;
+  void* win;
+  void* pool;
+};
+cudaError_t launch_decode_append(const DecodeAppendArgs& a, int dtype, cudaStream_t st);
+
 struct IndexerArgs {
   int B, Sq, nI, cI, m, P_cap, topk;
   const void* qI;

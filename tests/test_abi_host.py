@@ -123,6 +123,30 @@ def test_split_indexer_calls_reject_bad_arguments(abi):
     assert select(_params(abi, B=0)) == 0
 
 
+def test_decode_append_rejects_bad_arguments(abi):
+    lib = abi.load()
+
+    def call(p, c=512, apply_rope=1, **over):
+        a = dict(x=FAKE, z=FAKE, bias=FAKE, pos=FAKE, t=FAKE, buf_x=FAKE, buf_z=FAKE, buf_pos=FAKE, win=FAKE,
+                 pool=FAKE)
+        a.update(over)
+        return lib.dsv4_decode_append(ctypes.byref(p) if p is not None else None, c, a["x"], a["z"], a["bias"],
+                                      a["pos"], a["t"], a["buf_x"], a["buf_z"], a["buf_pos"], apply_rope,
+                                      a["win"], a["pool"], None)
+
+    assert call(None) == 1
+    assert call(_params(abi, win_ring=128), c=511) == 2                   # odd channel count
+    assert call(_params(abi, win_ring=128), t=None) == 1
+    assert call(_params(abi, win_ring=128), pos=None) == 1
+    assert call(_params(abi, win_ring=128), buf_z=None) == 1              # logits given but nowhere to buffer them
+    assert call(_params(abi, win_ring=0)) == 2              # a window ring of no rows
+    assert call(_params(abi, win_ring=128, R=63)) == 2                    # odd rope width
+    assert call(_params(abi, win_ring=128), apply_rope=2) == 1
+    assert call(_params(abi, win_ring=128), buf_x=FAKE + 4) == 3
+    assert call(_params(abi, win_ring=128, dtype=9)) == 4
+    assert call(_params(abi, win_ring=128, B=0)) == 0                     # nothing to append: no launch
+
+
 def test_compress_and_layers_reject_bad_arguments(abi):
     lib = abi.load()
     p = _params(abi)
