@@ -114,7 +114,7 @@ _ATTN_SOURCE = (("attn_tc.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
     # window 128): dram__bytes_read.sum 564.3 MB + dram__bytes_write.sum 494.1 MB.
-    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "75de456acf974ede70a65f460d38300dd361f15d3c325367bd5c59240c83f9ee", 1058375936),
+    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "838f7f5f3b791dfbdedc8b2b1af9b30e29dbb0721f5e6d77f66e8d1f3046a15a", 1058375936),
 }
 
 
