@@ -72,7 +72,7 @@ __device__ __forceinline__ float2 rope_pair(float2 v, int64_t pos, int d, int c,
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
+__global__ void __launch_bounds__(256, 5) compress_kernel(CompressArgs a) {
   const int w = blockIdx.x;
   const int b = blockIdx.y;
   const int c = a.c;

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cstddef>
 #include <cstdint>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -165,10 +166,6 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     ms->abort_flag = 0;
     tc::mbar_fence_init();
   }
-  if (warp == 4) {
-    tc::tmem_alloc(&ms->tmem_base, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
-    tc::tmem_relinquish();
-  }
   __syncthreads();
   // per-query visibility and head weights
   for (int q = tid; q < QB; q += kThreads) {
@@ -183,6 +180,19 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     atomicMax(&ms->maxvis, v);
   }
   for (int i = tid; i < 256 + 32; i += kThreads) ms->w[i] = (i < QB * nI && (i / nI) < nq) ? a.wI[rbase * nI + i] : 0.f;
+  __syncthreads();
+  // this CTA's entry tiles; a CTA past the group's visible entries leaves before loading
+  // anything (finer entry splits of causal prefill groups leave many such CTAs)
+  const int maxvis = ms->maxvis;
+  const int ntile_all = (maxvis + kTileE - 1) / kTileE;
+  const int t_lo = blockIdx.x * P.tiles_per_split;
+  const int t_hi = min(ntile_all, t_lo + P.tiles_per_split);
+  const int ntiles = t_hi > t_lo ? t_hi - t_lo : 0;
+  if (ntiles == 0) return;
+  if (warp == 4) {
+    tc::tmem_alloc(&ms->tmem_base, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
+    tc::tmem_relinquish();
+  }
   // (query, head) rows -> K-major 128B-swizzled B operand, by cp.async (rows past the group
   // are zero-filled with plain stores)
   {
@@ -206,11 +216,6 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
   __syncthreads();
   tc::tc_fence_after();
 
-  const int maxvis = ms->maxvis;
-  const int ntile_all = (maxvis + kTileE - 1) / kTileE;
-  const int t_lo = blockIdx.x * P.tiles_per_split;
-  const int t_hi = min(ntile_all, t_lo + P.tiles_per_split);
-  const int ntiles = t_hi > t_lo ? t_hi - t_lo : 0;
   const uint32_t tmem = ms->tmem_base;
   const uint32_t b_chunk = ((Npad * 128 + 1023) / 1024) * 1024;
 
@@ -378,8 +383,8 @@ cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r
   // scans about the whole pool: pick the tiles per CTA that minimise waves x (tiles per CTA
   // + a set-up cost of about two tiles), so that the last wave is not left mostly empty
   // (measured: 320 CTAs in 2.2 waves held the decode indexer to 63% of HBM bandwidth).
-  // Prefill (no cache indices) is causal: tile counts grow along the groups, and two splits
-  // per group once there are fewer groups than two waves balance it.
+  // Prefill (no cache indices) is causal: tile counts grow along the groups and are known
+  // here, so the same cost is evaluated over the CTAs that have work.
   const int nsm = indexer_num_sms();
   int best_tps = max_tiles;
   if (a.q_index) {
@@ -393,10 +398,27 @@ cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r
         best_tps = tps;
       }
     }
-  } else if (ngroups < 2 * nsm) {
-    int ns = (int)((2 * nsm + ngroups - 1) / ngroups);
-    if (ns > max_tiles) ns = max_tiles;
-    best_tps = (max_tiles + ns - 1) / ns;
+  } else {
+    // causal prefill: group g needs ceil(min((s0 + nq) / m, P_cap) / 128) tiles; CTAs past
+    // them exit at once, so the cost counts the non-empty CTAs only
+    std::vector<int64_t> groups_with(max_tiles + 1, 0);  // number of groups needing k tiles
+    for (int64_t g = g_lo; g < g_hi; ++g) {
+      const int gs0 = (int)(g % gps) * QB;
+      const int gnq = QB < a.Sq - gs0 ? QB : a.Sq - gs0;
+      int mv = (gs0 + gnq) / a.m;
+      if (mv > a.P_cap) mv = a.P_cap;
+      ++groups_with[(mv + kTileE - 1) / kTileE];
+    }
+    int64_t best_cost = INT64_MAX;
+    for (int tps = max_tiles; tps >= 1; --tps) {
+      int64_t n = 0;
+      for (int k = 1; k <= max_tiles; ++k) n += groups_with[k] * ((k + tps - 1) / tps);
+      const int64_t cost = ((n + nsm - 1) / nsm) * (tps + 2);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best_tps = tps;
+      }
+    }
   }
   P.tiles_per_split = best_tps;
   const int nsplit = (max_tiles + best_tps - 1) / best_tps;
