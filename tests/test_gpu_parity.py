@@ -342,3 +342,51 @@ def test_sliding_window_only_attention(lib, name, gains):
     g = _np(out)
     for b, s in rows:
         assert_max_abs(g[b, s], ref[b, s], ATTN_TOL[w.dtype], f"{name} window-only row {(b, s)}")
+
+
+def test_bench_step_path_csa_prefill(lib):
+    """The exact path bench.py times (harness.step_parts: the compressor, dsv4_indexer_scores
+    and dsv4_topk_select, the attention) at the full CSA prefill size, on sampled rows."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_prefill_bf16"]
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    o = harness.make_outputs(w, params, scores=True)
+    harness.step_parts(w, params, x, o)
+    abi.dsv4_device_check()
+    rows = [(0, s) for s in sample_rows(w.S, 192, 32)]
+    ref = O.csa_layer(host["q"], host["kv"], host["z"], host["bias"], host["qI"], host["wI"], host["kI"],
+                      host["zI"], host["biasI"], host["sink"], host["pos"], overlap=w.overlap, topk=w.topk,
+                      store="bf16", rows=rows, **_oracle_kw(w))
+    _check_layer_idx_and_out(w, host, o, ref, rows, rel_key_err=STORE_RTOL["bf16"])
+
+
+def test_bench_step_path_csa_decode(lib):
+    """The exact decode path bench.py times, at the full decode size (64 sequences, pool
+    32768, top-2048): top-k rows against the oracle's scores, attention rows whose
+    selection matches the oracle's."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_decode_bf16"]
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    o = harness.make_outputs(w, params, scores=True)
+    harness.step_parts(w, params, x, o)
+    abi.dsv4_device_check()
+    gidx, gout = _np(o["idx"]), _np(o["out"])
+    compared = 0
+    for b in range(0, w.B, 9):
+        t = int(host["q_index"][b, 0])
+        vis = O.visible_entries(t, w.m, w.P_cap)
+        sc = O.indexer_scores_row(host["qI"][b, 0], host["wI"][b, 0], host["poolI"][b], vis)
+        err = score_error_bound(host["qI"][b, 0], host["wI"][b, 0], host["poolI"][b][:vis], 0.0)
+        if check_topk_row(gidx[b, 0], sc, w.topk, err) == 0:
+            compared += 1
+            sel = gidx[b:b + 1, :1]
+            ref = O.sparse_mqa_attention(host["q"][b:b + 1], host["win"][b:b + 1], host["pool"][b:b + 1], sel,
+                                         host["sink"], host["qpos"][b:b + 1], host["q_index"][b:b + 1],
+                                         n_win=w.n_win, m=w.m, scale=w.scale, dv=w.dv, R=w.R, theta=w.theta,
+                                         rope_q=True, rotate_out=w.rotate_out, win_ring=w.win_ring, P_cap=w.P_cap)
+            assert_max_abs(gout[b, 0], ref[0, 0], ATTN_TOL[w.dtype], f"decode row {b}")
+    assert compared >= 5
