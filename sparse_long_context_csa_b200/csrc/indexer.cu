@@ -187,7 +187,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* 
 // selected prefix (skipped once the threshold digit holds exactly the keys still needed).
 // Output: the kept entries in ascending entry order, then -1.
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_kernel(IndexerArgs a, int64_t row0) {
+__global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs a, int64_t row0) {
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int wsum[NT / 32];
