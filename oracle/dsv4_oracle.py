@@ -40,6 +40,10 @@ its status:
   R6 output rotation: the rope slice of the output is rotated by -qpos (eq. 26)
      when the value width equals head_dim.  Pinned (shift invariance).
   R7 DSA (m=1, no window): a query sees tokens j <= t (itself included).
+  R13 sliding-window layers (`sliding_attention`): no pool and no indexer; keys
+     are the window rows only; their RoPE base is rope_theta (10000), since
+     compress_rope_theta belongs to the compressed layers.  Pinned (dense masked
+     attention with an empty compressor section).
 """
 from __future__ import annotations
 
@@ -59,6 +63,9 @@ __all__ = [
     "indexer_topk",
     "csa_layer",
     "hca_layer",
+    "sliding_layer",
+    "new_decode_cache",
+    "decode_append",
 ]
 
 
@@ -335,6 +342,19 @@ def hca_layer(q, kv, z, bias, sink, pos, *, m, n_win, scale, dv, R, theta, rotat
                                scale=scale, dv=dv, R=R, theta=theta, rope_q=True,
                                rotate_out=rotate_out, rows=rows)
     return {"pool": pool, "kv_rot": kv_rot, "out": out}
+
+
+def sliding_layer(q, kv, sink, pos, *, n_win, scale, dv, R, theta, rotate_out, rows=None, store=None):
+    """Prefill sliding-window layer ([V4] layer types, `sliding_attention`): no compressor
+    and no indexer; the K=V rows rotated at their positions, then attention over the
+    window (t - n_win, t] alone."""
+    B, S, D = kv.shape
+    kv_rot = store_as(rope_rotate(kv, pos, R, theta), store)
+    q_index = np.tile(np.arange(S), (B, 1))
+    out = sparse_mqa_attention(q, kv_rot, np.zeros((B, 0, D)), None, sink, pos, q_index, n_win=n_win, m=1,
+                               scale=scale, dv=dv, R=R, theta=theta, rope_q=True,
+                               rotate_out=rotate_out, P_cap=0, rows=rows)
+    return {"kv_rot": kv_rot, "out": out}
 
 
 # --------------------------------------------------------------------------

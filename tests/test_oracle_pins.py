@@ -318,6 +318,20 @@ def test_hca_equals_dense_masked_attention():
     np.testing.assert_allclose(res["out"][0], ref, atol=1e-12)
 
 
+def test_sliding_layer_equals_dense_window_attention():
+    """The window-only layer is the dense masked attention with an empty compressor section."""
+    x = _tiny_inputs(15, S=40)
+    kw = dict(n_win=7, scale=0.3, dv=16, R=8, theta=1000.0, rotate_out=1)
+    res = O.sliding_layer(x["q"], x["kv"], x["sink"], x["pos"], **kw)
+    ref = _dense_reference(x["q"], x["kv"], np.zeros((1, 0, 16)), x["sink"], x["pos"], m=1, **kw)
+    np.testing.assert_allclose(res["out"][0], ref, atol=1e-12)
+    # the first query sees only itself: softmax of one logit against the sink
+    qt = _rope_complex(x["q"][0, 0], 0, 8, 1000.0)
+    lg = 0.3 * qt @ x["kv"][0, 0]
+    p = 1.0 / (1.0 + np.exp(x["sink"] - lg))
+    np.testing.assert_allclose(res["out"][0, 0], p[:, None] * x["kv"][0, 0][None, :16], atol=1e-12)
+
+
 def test_csa_with_topk_covering_pool_equals_dense_masked_attention():
     x = _tiny_inputs(12, S=48, m=4, overlap=1)
     kw = dict(m=4, n_win=5, scale=0.3, dv=16, R=8, theta=1000.0, rotate_out=1)
