@@ -5,6 +5,10 @@
 A step is one pass of the whole hot path over one batch of synthetic input: for the
 default CSA prefill workload (B=1, S=8192, 64 heads, head_dim 512, m=4, top-512,
 window 128) that is compress(kv) + compress(kI) + indexer/top-k + sparse attention.
+Other workloads: HCA and DSA prefill, CSA decode over a pre-filled cache, a
+sliding-window layer (RoPE of the K=V rows + window attention) and the decode-cache
+append of one token per sequence (timed with L2 flushed between steps, since its
+inputs fit in L2).
 ``value`` is whole-job tokens/s with inputs resident in HBM (device time, CUDA events,
 max over ranks); ``e2e`` is the same metric through the layer entry point with pinned
 host inputs copied in and the output copied back every step.  With N > 1 every rank
@@ -64,9 +68,22 @@ def part_work(w, q_index):
     indexer_scores: visible entries x nI x cI x 2 FLOPs; bytes = the indexer pool once per
       sequence + qI + wI + the fp32 score rows written.
     topk: no FLOPs; bytes = the fp32 score rows read + the index rows written.
-    compress: bytes = token rows (kv and kI), logits and pools written.
+    compress: bytes = token rows (kv and kI) and their logits (m > 1) read, pools and the
+      rotated K=V rows written.
+    append: bytes per sequence and stream of c channels: the new row and its logits read and
+      written to the buffer (+ its position), the rotated window row (K=V stream); when the
+      token closes a block, the Lw buffered rows and logits read and the entry written.
     """
     e = 2 if w.dtype == "bf16" else 4
+    if w.kind == "append":
+        lw = 2 * w.m if w.overlap else w.m
+        t = q_index.reshape(-1).astype(np.int64)
+        closing = float(((t + 1) % w.m == 0).sum())
+        nbytes = 0.0
+        for c, window in ((w.D, True), (w.cI, False)):
+            nbytes += w.B * (4 * c * e + 8 + (c * e if window else 0))
+            nbytes += closing * (2 * lw * c * e + lw * c * 4 + c * e)
+        return {"append": (0.0, nbytes)}
     nq = w.B * w.Sq
     keys = float(attn_keys_per_query(w, q_index).sum())
     vis = _visible(w, q_index).astype(np.float64)
@@ -83,7 +100,8 @@ def part_work(w, q_index):
         work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
     if w.kind != "decode":
         ch = w.D + (w.cI if w.nI else 0)
-        work["compress"] = (0.0, w.B * w.S * ch * e * 2 + w.B * w.P_cap * ch * e + w.B * w.S * w.D * e)
+        rows_in = w.B * w.S * ch * e * (2 if w.m > 1 else 1)
+        work["compress"] = (0.0, rows_in + w.B * w.P_cap * ch * e + w.B * w.S * w.D * e)
     return work
 
 
@@ -224,9 +242,35 @@ def cpu_oracle_rate(w, budget_s: float, host=None):
                 break
         dt = time.perf_counter() - t0
         return done / dt, done, dt, f"{done} of {w.B} decode sequences (indexer + top-k + attention)"
+    if w.kind == "append":
+        # per sequence: the Lw-1 earlier tokens are appended untimed, the step's token timed
+        lw = host["kv"].shape[0]
+        done, dt = 0, 0.0
+        for b in range(w.B):
+            caches = [(O.new_decode_cache(w.D, m=w.m, overlap=w.overlap, P_cap=w.P_cap, win_ring=w.win_ring),
+                       "kv", "z", "bias", True),
+                      (O.new_decode_cache(w.cI, m=w.m, overlap=w.overlap, P_cap=w.P_cap), "kI", "zI", "biasI", False)]
+            for k in range(lw):
+                if k == lw - 1:
+                    t1 = time.perf_counter()
+                for cache, xk, zk, bk, rope in caches:
+                    O.decode_append(cache, host[xk][k, b], host[zk][k, b], int(host["pos_hist"][k, b]),
+                                    int(host["t_hist"][k, b]), m=w.m, overlap=w.overlap, bias=host[bk],
+                                    apply_rope=rope, R=w.R, theta=w.theta)
+            dt += time.perf_counter() - t1
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        return done / dt, done, time.perf_counter() - t0, (
+            f"{done} of {w.B} sequences: one token appended to the K=V and indexer-key caches "
+            f"(the {lw - 1} tokens before it appended untimed)")
     kw = dict(m=w.m, n_win=w.n_win, scale=w.scale, dv=w.dv, R=w.R, theta=w.theta, rotate_out=w.rotate_out)
-    pool = O.compress(host["kv"], host.get("z"), host.get("bias"), host["pos"], m=w.m, overlap=w.overlap,
-                      apply_rope=True, R=w.R, theta=w.theta)
+    if w.kind == "swa":
+        pool = np.zeros((w.B, 0, w.D))
+        kw["P_cap"] = 0
+    else:
+        pool = O.compress(host["kv"], host.get("z"), host.get("bias"), host["pos"], m=w.m, overlap=w.overlap,
+                          apply_rope=True, R=w.R, theta=w.theta)
     kv_rot = O.rope_rotate(host["kv"], host["pos"], w.R, w.theta)
     poolI = O.compress(host["kI"], host.get("zI"), host.get("biasI"), host["pos"], m=w.m,
                        overlap=w.overlap, apply_rope=False) if w.nI > 0 else None
@@ -247,8 +291,9 @@ def cpu_oracle_rate(w, budget_s: float, host=None):
     t_rows = time.perf_counter() - t1
     per_row = t_rows / max(done, 1)
     total = t_comp + per_row * w.S * w.B
+    first = "RoPE of all" if w.kind == "swa" else "compression of all"
     return (w.S * w.B) / total, done, t_comp + t_rows, (
-        f"compression of all {w.S} tokens ({t_comp:.2f} s) + {done} random query rows "
+        f"{first} {w.S} tokens ({t_comp:.2f} s) + {done} random query rows "
         f"({per_row * 1e3:.1f} ms/row), extrapolated to {w.S} rows")
 
 
@@ -272,7 +317,7 @@ def run_reference(args, w):
         rate, rows, secs, desc = cpu_oracle_rate(w, args.ref_budget, host)
         if i >= args.warmup:
             per_step.append(rate)
-    if w.kind == "decode":
+    if per_step_kind(w) == "us/step":
         value = 1e6 / float(np.mean(per_step)) * w.B  # us per step of all B sequences
         unit = "us/step"
     else:
@@ -299,12 +344,26 @@ def reduce_max(v: float, world: int, device: str) -> float:
     return float(t.item())
 
 
+def per_step_kind(w) -> str:
+    """Decode workloads (one token per sequence) report us/step, prefill ones tokens/s."""
+    return "us/step" if w.kind in ("decode", "append") else "tokens/s"
+
+
 def job_value(kind: str, world: int, tokens_per_rank: int, steps: int, ms_max: float):
     """Whole-job metric from the slowest rank's time for `steps` steps: decode reports
     microseconds per step; prefill reports the tokens of all ranks per second."""
-    if kind == "decode":
+    if kind in ("decode", "append"):
         return ms_max / steps * 1e3, "us/step", False
     return world * tokens_per_rank * steps / (ms_max / 1e3), "tokens/s", True
+
+
+def l2_flush_needed(w) -> bool:
+    """True when a step's inputs fit in the 126 MB L2: such steps are timed with L2 flushed."""
+    if w.kind == "append":
+        return True
+    if w.kind == "decode":
+        return w.B * w.P_cap * (w.D + w.cI) * 2 <= (126 << 20)
+    return w.B * w.Sq * w.H * w.D * 2 <= (126 << 20)
 
 
 def config_of(w):
@@ -312,8 +371,16 @@ def config_of(w):
          "dv": w.dv, "sliding_window": w.n_win, "m": w.m, "overlap": w.overlap, "pool_cap": w.P_cap}
     if w.nI:
         c.update({"index_n_heads": w.nI, "index_head_dim": w.cI, "index_topk": w.topk})
-    c["l2"] = "inputs larger than L2 (q and out are each > 126 MB)" if w.B * w.Sq * w.H * w.D * 2 > (126 << 20) \
-        else "L2 flushed between steps"
+    if w.kind == "append":
+        c = {"workload": w.name, "B": w.B, "cache_tokens": w.S, "head_dim": w.D, "rope_dim": w.R, "m": w.m,
+             "overlap": w.overlap, "buffer_rows": 2 * w.m if w.overlap else w.m, "window_ring": w.win_ring,
+             "pool_cap": w.P_cap, "index_head_dim": w.cI}
+    if l2_flush_needed(w):
+        c["l2"] = "L2 flushed between steps (a 256 MiB buffer written outside the timed events)"
+    elif w.kind == "decode":
+        c["l2"] = "inputs larger than L2 (pools 2.5 GB)"
+    else:
+        c["l2"] = "inputs larger than L2 (q and out are each > 126 MB)"
     return c
 
 
@@ -365,6 +432,10 @@ def main():
     def step(events=None):
         harness.step_parts(w, params, x, o, stream, events=events)
 
+    if w.kind == "append":
+        harness.append_prefill(w, params, x, o, stream)  # the cache just before the step's token
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if l2_flush_needed(w) else None
+
     # warm-up (also starts the clock sampler and lets it settle)
     sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
     if not args.profile_run:
@@ -381,19 +452,27 @@ def main():
     evs = [{p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for p in parts}
            for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)] if flush is not None else None
     barrier()
     torch.cuda.synchronize()
     n0 = abi.dsv4_launch_count()
     wall0 = time.time()
     start.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 255)  # evicts the previous step's lines from L2; not inside the step's events
+            step_ev[i][0].record(stream)
         step(evs[i])
+        if flush is not None:
+            step_ev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
     n1 = abi.dsv4_launch_count()
     barrier()
-    ms = max_over_ranks(start.elapsed_time(end))
+    total_ms = start.elapsed_time(end) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
+    ms = max_over_ranks(total_ms)
     part_ms = {p: max_over_ranks(float(np.mean([e[p][0].elapsed_time(e[p][1]) for e in evs]))) for p in parts}
     clocks = sampler.summary(wall0, wall1)
     if args.profile_run:
@@ -403,16 +482,25 @@ def main():
 
     # end to end through the layer entry point: pinned host inputs in, output back
     host_t = harness.to_device(w, host, device=None, pin=True)
-    out_host = torch.empty(o["out"].shape, dtype=o["out"].dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in host_t.values())
+    if w.kind == "append":
+        # the step's token (rows, logits, position, cache index) in; the buffer's position
+        # record back (the rows themselves stay on the device for attention)
+        last = host["kv"].shape[0] - 1
+        pairs = [(x[k][last], host_t[k][last]) for k in ("kv", "z", "kI", "zI", "pos_hist", "t_hist")]
+        result = o["buf_pos"]
+    else:
+        pairs = [(x[k], t) for k, t in host_t.items()]
+        result = o["out"]
+    out_host = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for _, t in pairs)
     d2h = out_host.numel() * out_host.element_size()
     e2e_steps = max(3, min(args.steps, 10))
 
     def e2e_step():
-        for k, t in host_t.items():
-            x[k].copy_(t, non_blocking=True)
+        for dst, src in pairs:
+            dst.copy_(src, non_blocking=True)
         harness.step(w, params, x, o, stream)
-        out_host.copy_(o["out"], non_blocking=True)
+        out_host.copy_(result, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -448,7 +536,7 @@ def main():
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, rows, secs, desc = cpu_oracle_rate(w, args.cpu_budget, host)
-        cv = (1e6 / rate * w.B) if w.kind == "decode" else rate
+        cv = (1e6 / rate * w.B) if per_step_kind(w) == "us/step" else rate
         line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": blas_threads(), "kind": "oracle",
                                 "sample": desc, "seconds": round(secs, 2)}
     if rank == 0:

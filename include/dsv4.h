@@ -99,6 +99,8 @@ typedef struct dsv4_params {
  *   pos    [B,S] int64        RoPE positions (required when apply_rope)
  *   pool   [B,P_cap,c] T      out: entries 0 .. S/m-1 are written (S/m <= P_cap)
  *   x_rot  [B,S,c] T or NULL  out: x rotated at pos (the window keys); needs apply_rope
+ * A sliding-window layer ([V4] layer types, `sliding_attention`) keeps no pool: with
+ * P_cap == 0 and pool == NULL the call only writes x_rot (which is then required).
  */
 dsv4_status dsv4_compress_kv(const dsv4_params* params, int32_t c, const void* x, const void* z,
                              const float* bias, const int64_t* pos, int32_t apply_rope,

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256, 5) compress_kernel(CompressArgs a) {
   const T* __restrict__ z = a.z ? static_cast<const T*>(a.z) + (int64_t)b * S * c : nullptr;
   const int64_t* pos = a.pos ? a.pos + (int64_t)b * S : nullptr;
 
-  if (w < P) {
+  if (a.pool && w < P) {
     const int lo = a.overlap ? (w - 1) * m : w * m;
     const int hi = (w + 1) * m;
     const int j0 = lo < 0 ? 0 : lo;

@@ -88,8 +88,10 @@ dsv4_status from_cuda(cudaError_t e) {
 dsv4_status run_compress(const dsv4_params* p, int c, const void* x, const void* z, const float* bias,
                          const int64_t* pos, int apply_rope, void* pool, void* x_rot, void* stream) {
   if (c < 2 || (c & 1)) return DSV4_ERR_SHAPE;
-  if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
-  if (!ok_ptr(x) || !ok_ptr(pool)) return x && pool ? DSV4_ERR_ALIGN : DSV4_ERR_ARG;
+  const bool rotate_only = pool == nullptr && p->P_cap == 0;  // sliding-window layer: no pool
+  if (!rotate_only && p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
+  if (!x || (!pool && !rotate_only) || (rotate_only && !x_rot)) return DSV4_ERR_ARG;
+  if (!ok_ptr(x) || (pool && !aligned16(pool))) return DSV4_ERR_ALIGN;
   if ((z && !aligned16(z)) || (bias && !aligned16(bias)) || (x_rot && !aligned16(x_rot))) return DSV4_ERR_ALIGN;
   if (apply_rope != 0 && apply_rope != 1) return DSV4_ERR_ARG;
   if (apply_rope) {

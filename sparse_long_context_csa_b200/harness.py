@@ -4,6 +4,10 @@ A "step" is one pass of the hot path over one batch:
   prefill CSA / DSA: dsv4_csa_layer (compress kv, compress kI, indexer + top-k, attention)
   prefill HCA:       dsv4_hca_layer (compress kv, attention over every visible entry)
   decode:            dsv4_indexer_topk + dsv4_sparse_mqa_attn over a pre-filled cache
+  sliding window:    dsv4_compress_kv without a pool (RoPE of the K=V rows) +
+                     dsv4_sparse_mqa_attn over the window alone
+  decode append:     dsv4_decode_append of one token per sequence to the K=V stream
+                     (buffer, window ring, pool) and to the indexer-key stream
 PyTorch only allocates device memory and supplies the stream; every step of the
 method runs inside libdsv4.
 """
@@ -56,11 +60,29 @@ def to_device(w, host: dict, device="cuda", pin=False) -> dict:
     return out
 
 
+def append_state(w, device="cuda") -> dict:
+    """Decode-cache state of both streams of a workload of kind "append", zero-filled: the
+    compressor buffers (Lw rows, their logits and positions), the K=V window ring and the
+    two pools."""
+    dt = torch_dtype(w)
+    lw = 2 * w.m if w.overlap else w.m
+
+    def z(*shape, dtype=dt):
+        return torch.zeros(shape, dtype=dtype, device=device)
+
+    return {"buf_x": z(w.B, lw, w.D), "buf_z": z(w.B, lw, w.D), "buf_pos": z(w.B, lw, dtype=torch.int64),
+            "bufI_x": z(w.B, lw, w.cI), "bufI_z": z(w.B, lw, w.cI), "bufI_pos": z(w.B, lw, dtype=torch.int64),
+            "win": z(w.B, w.win_ring, w.D), "pool": z(w.B, w.P_cap, w.D), "poolI": z(w.B, w.P_cap, w.cI)}
+
+
 def make_outputs(w, params: abi.Dsv4Params, device="cuda", scores=False) -> dict:
     dt = torch_dtype(w)
+    if w.kind == "append":
+        return append_state(w, device)
     o = {"out": torch.empty((w.B, w.Sq, w.H, w.dv), dtype=dt, device=device)}
     if w.kind != "decode":
-        o["pool"] = torch.empty((w.B, w.P_cap, w.D), dtype=dt, device=device)
+        if w.P_cap > 0:
+            o["pool"] = torch.empty((w.B, w.P_cap, w.D), dtype=dt, device=device)
         o["kv_rot"] = torch.empty((w.B, w.S, w.D), dtype=dt, device=device)
     if w.nI > 0:
         if w.kind != "decode":
@@ -73,8 +95,28 @@ def make_outputs(w, params: abi.Dsv4Params, device="cuda", scores=False) -> dict
     return o
 
 
+def append_token(w, params, x: dict, o: dict, k: int, stream=None) -> None:
+    """Append history token k (rows x["kv"][k], x["kI"][k], ...) to every sequence's cache:
+    the K=V stream (rotated window row; entry pooled and rotated when the token closes a
+    block) and the indexer-key stream (no RoPE, no window)."""
+    abi.dsv4_decode_append(params, w.D, x["kv"][k], x["z"][k], x["bias"], x["pos_hist"][k], x["t_hist"][k],
+                           o["buf_x"], o["buf_z"], o["buf_pos"], 1, o["win"], o["pool"], stream=stream)
+    abi.dsv4_decode_append(params, w.cI, x["kI"][k], x["zI"][k], x["biasI"], x["pos_hist"][k], x["t_hist"][k],
+                           o["bufI_x"], o["bufI_z"], o["bufI_pos"], 0, None, o["poolI"], stream=stream)
+
+
+def append_prefill(w, params, x: dict, o: dict, stream=None) -> None:
+    """Bring the cache to the state just before the step's token: append the Lw-1 tokens
+    before it, so that the buffers hold every token that the step's pooling reads."""
+    for k in range(x["kv"].shape[0] - 1):
+        append_token(w, params, x, o, k, stream)
+
+
 def step(w, params, x: dict, o: dict, stream=None) -> None:
     """Enqueue one step of the workload's hot path (see module docstring)."""
+    if w.kind == "append":
+        append_token(w, params, x, o, x["kv"].shape[0] - 1, stream)
+        return
     ws = o["workspace"]
     if w.kind in ("csa", "dsa"):
         abi.dsv4_csa_layer(params, x["q"], x["kv"], x.get("z"), x.get("bias"), x["qI"], x["wI"], x["kI"],
@@ -87,11 +129,13 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
         abi.dsv4_indexer_topk(params, x["qI"], x["wI"], x["poolI"], x["q_index"], o["idx"], ws, stream=stream)
         abi.dsv4_sparse_mqa_attn(params, x["q"], x["win"], x["pool"], o["idx"], x["sink"], x["qpos"],
                                  x["q_index"], o["out"], ws, stream=stream)
+    elif w.kind == "swa":
+        step_parts(w, params, x, o, stream)
     else:
         raise ValueError(w.kind)
 
 
-PARTS = ("compress", "indexer_scores", "topk", "attention")
+PARTS = ("append", "compress", "indexer_scores", "topk", "attention")
 
 
 def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
@@ -99,17 +143,22 @@ def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
     halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select): the same
     kernels on the same data.  ``events`` maps names of ``PARTS`` to (start, end) CUDA
     event pairs recorded on ``stream`` around that part."""
-    ws = o["workspace"]
+    ws = o.get("workspace")
 
     def mark(name, k):
         if events is not None and name in events:
             events[name][k].record(stream)
 
-    if w.kind in ("csa", "dsa", "hca"):
+    if w.kind == "append":
+        mark("append", 0)
+        step(w, params, x, o, stream)
+        mark("append", 1)
+        return
+    if w.kind in ("csa", "dsa", "hca", "swa"):
         mark("compress", 0)
-        abi.dsv4_compress_kv(params, w.D, x["kv"], x.get("z"), x.get("bias"), x["pos"], 1, o["pool"],
+        abi.dsv4_compress_kv(params, w.D, x["kv"], x.get("z"), x.get("bias"), x["pos"], 1, o.get("pool"),
                              o["kv_rot"], stream=stream)
-        if w.kind != "hca":
+        if w.kind in ("csa", "dsa"):
             abi.dsv4_compress_kv(params, w.cI, x["kI"], x.get("zI"), x.get("biasI"), None, 0, o["poolI"], None,
                                  stream=stream)
         mark("compress", 1)
@@ -127,6 +176,6 @@ def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
         abi.dsv4_sparse_mqa_attn(params, x["q"], x["win"], x["pool"], o["idx"], x["sink"], x["qpos"],
                                  x["q_index"], o["out"], ws, stream=stream)
     else:
-        abi.dsv4_sparse_mqa_attn(params, x["q"], o["kv_rot"], o["pool"], o.get("idx") if w.kind != "hca" else None,
-                                 x["sink"], x["pos"], None, o["out"], ws, stream=stream)
+        abi.dsv4_sparse_mqa_attn(params, x["q"], o["kv_rot"], o.get("pool"), o.get("idx"), x["sink"], x["pos"],
+                                 None, o["out"], ws, stream=stream)
     mark("attention", 1)

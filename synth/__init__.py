@@ -31,13 +31,14 @@ STREAMS = {
     "q": 1, "kv": 2, "z": 3, "bias": 4, "qI": 5, "wI": 6, "kI": 7, "zI": 8,
     "biasI": 9, "sink": 10, "pool": 11, "poolI": 12, "win": 13, "q_index": 14,
 }
+# (stream 15 draws the offsets of strided_selection)
 
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
     config_id: int
-    kind: str            # "csa" | "hca" | "decode" | "dsa"
+    kind: str            # "csa" | "hca" | "decode" | "dsa" | "swa" (window only) | "append"
     dtype: str           # "f32" | "bf16"
     B: int
     S: int               # tokens in the sequence (prefill) / cache length (decode)
@@ -87,6 +88,17 @@ WORKLOADS = {
     "dsa_prefill_bf16": Workload("dsa_prefill_bf16", 4, "dsa", "bf16", B=1, S=32768, Sq=32768,
                                  H=64, D=576, R=64, dv=512, n_win=0, m=1, overlap=0, nI=1,
                                  cI=128, topk=2048, theta=10000.0, rotate_out=0, P_cap=32768),
+    # a sliding_attention layer of the same shape as the CSA prefill: RoPE of the K=V rows,
+    # then attention over the 128-token window alone (no pool, no indexer)
+    "swa_prefill_bf16": Workload("swa_prefill_bf16", 5, "swa", "bf16", B=1, S=8192, Sq=8192,
+                                 H=64, D=512, R=64, dv=512, n_win=128, m=1, overlap=0, nI=0,
+                                 cI=0, topk=0, theta=10000.0, rotate_out=1, P_cap=0),
+    # one decode-cache append per sequence of the CSA decode cache: the K=V stream (buffer,
+    # window ring, pool) and the indexer-key stream (buffer, pool)
+    "csa_decode_append_bf16": Workload("csa_decode_append_bf16", 6, "append", "bf16", B=64, S=131072,
+                                       Sq=1, H=64, D=512, R=64, dv=512, n_win=128, m=4, overlap=1,
+                                       nI=8, cI=128, topk=2048, theta=160000.0, rotate_out=1,
+                                       P_cap=32768, win_ring=128, qindex_spread=1024),
 }
 
 
@@ -171,6 +183,16 @@ def tensor_specs(w: Workload, gains: dict | None = None) -> dict:
     def spec(name, shape, scale, bf16=bf):
         return TensorSpec(s, STREAMS[name], tuple(shape), float(scale) * gains.get(name, 1.0), bf16)
 
+    if w.kind == "append":
+        # rows of the last Lw tokens of every sequence, token-major ([Lw, B, c]); the last
+        # one is the token the step appends
+        lw = 2 * w.m if w.overlap else w.m
+        return {"kv": spec("kv", (lw * w.B, w.D), 1 / math.sqrt(w.D)),
+                "z": spec("z", (lw * w.B, w.D), 1.0),
+                "bias": spec("bias", (lw, w.D), 0.1, bf16=False),
+                "kI": spec("kI", (lw * w.B, w.cI), 1 / math.sqrt(w.cI)),
+                "zI": spec("zI", (lw * w.B, w.cI), 1.0),
+                "biasI": spec("biasI", (lw, w.cI), 0.1, bf16=False)}
     specs = {
         "q": spec("q", (w.B * w.Sq, w.H, w.D), 1 / math.sqrt(w.D)),
         "sink": spec("sink", (w.H,), 1.0, bf16=False),
@@ -203,7 +225,7 @@ def positions(w: Workload) -> tuple[np.ndarray, np.ndarray]:
     Prefill: query s sits at cache index s.  Decode: each sequence's new token
     sits at S-1-U{0..qindex_spread-1}, drawn from stream ``q_index``.
     """
-    if w.kind == "decode":
+    if w.kind in ("decode", "append"):
         rng = np.random.default_rng([w.seed, STREAMS["q_index"], 0])
         qi = (w.S - 1 - rng.integers(0, w.qindex_spread, size=(w.B, 1))).astype(np.int64)
     else:
@@ -218,6 +240,8 @@ def token_positions(w: Workload) -> np.ndarray:
 
 def reshape(w: Workload, name: str, a: np.ndarray) -> np.ndarray:
     """Unflatten a full tensor drawn from ``tensor_specs`` to its logical shape."""
+    if w.kind == "append":
+        return a.reshape((-1, w.B) + a.shape[1:]) if name in ("kv", "z", "kI", "zI") else a
     shapes = {
         "q": (w.B, w.Sq, w.H, w.D), "kv": (w.B, w.S, w.D), "z": (w.B, w.S, w.D),
         "qI": (w.B, w.Sq, w.nI, w.cI), "wI": (w.B, w.Sq, w.nI), "kI": (w.B, w.S, w.cI),
@@ -231,7 +255,13 @@ def make_inputs(w: Workload, gains: dict | None = None, threads: int = 8) -> dic
     """All inputs of ``w`` as float32 numpy arrays in their logical shapes, plus positions."""
     out = {name: reshape(w, name, sp.full(threads)) for name, sp in tensor_specs(w, gains).items()}
     out["q_index"], out["qpos"] = positions(w)
-    if w.kind != "decode":
+    if w.kind == "append":
+        # cache index (= position) of history token k of sequence b: q_index[b] - (Lw-1-k)
+        lw = out["kv"].shape[0]
+        t = out["q_index"][:, 0][None, :] - np.arange(lw - 1, -1, -1, dtype=np.int64)[:, None]
+        out["t_hist"] = t.astype(np.int32)
+        out["pos_hist"] = t.astype(np.int64)
+    elif w.kind != "decode":
         out["pos"] = token_positions(w)
     return out
 

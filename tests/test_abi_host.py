@@ -155,6 +155,15 @@ def test_compress_and_layers_reject_bad_arguments(abi):
     assert lib.dsv4_compress_kv(ctypes.byref(p), 512, FAKE, None, None, FAKE, 0, FAKE, FAKE, None) == 1
     small = _params(abi, P_cap=100)  # S/m = 2048 entries do not fit
     assert lib.dsv4_compress_kv(ctypes.byref(small), 512, FAKE, None, None, FAKE, 1, FAKE, None, None) == 2
+    # sliding-window layers: no pool (P_cap 0, pool NULL) -> only the rotated rows, which are required
+    nopool = _params(abi, P_cap=0)
+    assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE, None, None, FAKE, 1, None, None, None) == 1
+    assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE, None, None, FAKE, 0, None, FAKE, None) == 1
+    assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE, None, None, FAKE, 1, FAKE, FAKE, None) == 2
+    assert lib.dsv4_compress_kv(ctypes.byref(p), 512, FAKE, None, None, FAKE, 1, None, FAKE, None) == 1
+    assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE + 4, None, None, FAKE, 1, None, FAKE, None) == 3
+    assert lib.dsv4_compress_kv(ctypes.byref(_params(abi, P_cap=0, B=0)), 512, FAKE, None, None, FAKE, 1, None,
+                                FAKE, None) == 0
     args = [FAKE] * 17  # q .. idx, workspace
     assert lib.dsv4_csa_layer(ctypes.byref(_params(abi, Sq=1)), *args, 1 << 40, None) == 2   # prefill only
     assert lib.dsv4_csa_layer(ctypes.byref(p), *args, 16, None) == 7                          # workspace too small

@@ -97,3 +97,57 @@ def test_decode_append_matches_prefill_compression(lib, name, stream):
         for j in range(S - ring, S):
             assert_close_rel(gw[:, j % ring], rot[:, j], STORE_RTOL[w.dtype], 4 * U32 * float(np.abs(x).max()),
                              f"window row {j}")
+
+
+def test_bench_step_path_decode_append(lib):
+    """The decode-cache append bench.py times, at full size (64 sequences, pool 32768, window
+    ring 128, K=V and indexer-key streams): the Lw-1 earlier tokens and then the step's token
+    are appended to zeroed caches on both sides.  Every sequence's window slot holds its
+    rotated token; every entry closed on the way matches the oracle's; the buffered positions
+    are exact; repeating the step changes no bit."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_decode_append_bf16"]
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    o = harness.make_outputs(w, params)
+    harness.append_prefill(w, params, x, o)
+    harness.step_parts(w, params, x, o)
+    abi.dsv4_device_check()
+    lw = host["kv"].shape[0]
+    t_last = host["t_hist"][-1].astype(np.int64)
+    bidx = torch.arange(w.B, device="cuda")
+    wslot = torch.from_numpy(t_last % w.win_ring).cuda()
+    closes = [(k, b) for k in range(lw) for b in range(w.B) if (int(host["t_hist"][k, b]) + 1) % w.m == 0]
+    eb = torch.tensor([b for _, b in closes], device="cuda")
+    ew = torch.tensor([(int(host["t_hist"][k, b]) + 1) // w.m - 1 for k, b in closes], device="cuda")
+    before = (o["win"][bidx, wslot].clone(), o["buf_x"].clone(), o["buf_pos"].clone(), o["pool"][eb, ew].clone(),
+              o["poolI"][eb, ew].clone())
+    harness.step(w, params, x, o)   # the timed step once more: the same slots, the same bits
+    abi.dsv4_device_check()
+    after = (o["win"][bidx, wslot], o["buf_x"], o["buf_pos"], o["pool"][eb, ew], o["poolI"][eb, ew])
+    for u, v in zip(before, after):
+        assert torch.equal(u, v), "repeating the append changed the cache"
+
+    g_win = before[0].float().cpu().numpy()
+    g_pos = before[2].cpu().numpy()
+    g_pool = {(k, b): r for (k, b), r in zip(closes, before[3].float().cpu().numpy())}
+    g_poolI = {(k, b): r for (k, b), r in zip(closes, before[4].float().cpu().numpy())}
+    kw = dict(m=w.m, overlap=w.overlap, R=w.R, theta=w.theta)
+    for b in range(w.B):
+        kvc = O.new_decode_cache(w.D, m=w.m, overlap=w.overlap, P_cap=w.P_cap, win_ring=w.win_ring)
+        kic = O.new_decode_cache(w.cI, m=w.m, overlap=w.overlap, P_cap=w.P_cap)
+        for k in range(lw):
+            t, pos = int(host["t_hist"][k, b]), int(host["pos_hist"][k, b])
+            O.decode_append(kvc, host["kv"][k, b], host["z"][k, b], pos, t, bias=host["bias"], apply_rope=True, **kw)
+            O.decode_append(kic, host["kI"][k, b], host["zI"][k, b], pos, t, bias=host["biasI"], apply_rope=False,
+                            **kw)
+            if (t + 1) % w.m == 0:
+                e = (t + 1) // w.m - 1
+                assert_close_rel(g_pool[(k, b)], kvc["pool"][e], STORE_RTOL["bf16"],
+                                 (lw + 8) * U32 * float(np.abs(host["kv"]).max()), f"K=V entry {e} of seq {b}")
+                assert_close_rel(g_poolI[(k, b)], kic["pool"][e], STORE_RTOL["bf16"],
+                                 (lw + 8) * U32 * float(np.abs(host["kI"]).max()), f"indexer entry {e} of seq {b}")
+        assert_close_rel(g_win[b], kvc["win"][t_last[b] % w.win_ring], STORE_RTOL["bf16"],
+                         4 * U32 * float(np.abs(host["kv"]).max()), f"window row of seq {b}")
+        np.testing.assert_array_equal(g_pos[b], kvc["pos"])

@@ -390,3 +390,27 @@ def test_bench_step_path_csa_decode(lib):
                                          rope_q=True, rotate_out=w.rotate_out, win_ring=w.win_ring, P_cap=w.P_cap)
             assert_max_abs(gout[b, 0], ref[0, 0], ATTN_TOL[w.dtype], f"decode row {b}")
     assert compared >= 5
+
+
+def test_bench_step_path_swa_prefill(lib):
+    """The sliding-window layer bench.py times, at full size (B=1, S=8192, 64 heads, window
+    128): RoPE of the K=V rows with no pool (rotated rows within one storage ulp of the
+    oracle's), then attention over the window alone (sampled rows within the attention
+    tolerance of the oracle's sliding layer, which reads the same bf16-stored rows)."""
+    abi, harness = lib
+    w = synth.WORKLOADS["swa_prefill_bf16"]
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    o = harness.make_outputs(w, params, scores=True)
+    assert "pool" not in o and "idx" not in o
+    harness.step_parts(w, params, x, o)
+    abi.dsv4_device_check()
+    rot = O.rope_rotate(host["kv"], host["pos"], w.R, w.theta)
+    assert_close_rel(_np(o["kv_rot"]), rot, STORE_RTOL["bf16"], fp32_atol(host["kv"], 4), "rotated K=V rows")
+    rows = [(0, s) for s in sample_rows(w.S, 192, 32)]
+    ref = O.sliding_layer(host["q"], host["kv"], host["sink"], host["pos"], n_win=w.n_win, scale=w.scale,
+                          dv=w.dv, R=w.R, theta=w.theta, rotate_out=w.rotate_out, rows=rows, store="bf16")
+    g = _np(o["out"])
+    for b, s in rows:
+        assert_max_abs(g[b, s], ref["out"][b, s], ATTN_TOL["bf16"], f"window-only row {s}")
