@@ -126,57 +126,115 @@ cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st) {
 // Decode-cache append: one CTA per sequence, thread per channel pair.  The new token goes to
 // buffer slot t % Lw (raw row, logits, position) and, rotated, to window-ring slot
 // t % win_ring; when it closes a block, the entry of that block is pooled from the buffer.
-// A thread reads back only the channels it wrote itself; the buffered positions, written by
-// thread 0, are read after a barrier.
-template <typename T>
+//
+// The kernel is latency-bound (a few hundred bytes per sequence), so it is built around
+// memory round trips.  When the buffer fits in shared memory (kStaged: Lw x c rows of x, z
+// and the fp32 bias, plus Lw positions), every read the step can need (the cache index, the
+// new row, all Lw buffered rows, the bias, the buffered positions) is issued at once, before
+// the cache index is known (no address depends on it), into shared memory; the entry is then
+// pooled from there: one round trip instead of four.  Otherwise the buffer is pooled in place
+// (the buffered positions, written by thread 0, are read after a barrier).  Both paths pool
+// with pool_pair, so the entry has the same bits as the one the prefill compressor writes.
+template <typename T, bool kStaged>
 __global__ void __launch_bounds__(256) decode_append_kernel(DecodeAppendArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
   const int b = blockIdx.x;
-  const int t = a.t[b];
-  if (t < 0) return;
   const int c = a.c, m = a.m;
   const int lw = a.overlap ? 2 * m : m;
+  const int t = a.t[b];
   const int64_t pos = a.pos[b];
   const T* __restrict__ xn = static_cast<const T*>(a.x) + (int64_t)b * c;
   const T* __restrict__ zn = a.z ? static_cast<const T*>(a.z) + (int64_t)b * c : nullptr;
   T* __restrict__ bx = static_cast<T*>(a.buf_x) + (int64_t)b * lw * c;
   T* __restrict__ bz = a.buf_z ? static_cast<T*>(a.buf_z) + (int64_t)b * lw * c : nullptr;
-  const int slot = t % lw;
+  int64_t* __restrict__ bpos = a.buf_pos + (int64_t)b * lw;
+
+  // where the pooling reads the buffer: in place, or the shared-memory copy
+  T* px = bx;
+  T* pz = bz;
+  const float* pb = a.bias;
+  int64_t* ppos = bpos;
+  if constexpr (kStaged) {
+    px = reinterpret_cast<T*>(sm);
+    pz = bz ? px + lw * c : nullptr;
+    float* sb = reinterpret_cast<float*>(px + 2 * lw * c);
+    ppos = reinterpret_cast<int64_t*>(sb + lw * c);
+    for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
+#pragma unroll 8
+      for (int r = 0; r < lw; ++r) {
+        const float2 xv = load2<T>(bx + (int64_t)r * c + d);
+        store2<T>(px + r * c + d, xv.x, xv.y);
+        if (bz) {
+          const float2 zv = load2<T>(bz + (int64_t)r * c + d);
+          store2<T>(pz + r * c + d, zv.x, zv.y);
+        }
+        if (a.bias) *reinterpret_cast<float2*>(sb + r * c + d) = *reinterpret_cast<const float2*>(a.bias + r * c + d);
+      }
+    }
+    if (a.bias) pb = sb;
+    for (int r = threadIdx.x; r < lw; r += blockDim.x) ppos[r] = bpos[r];
+  }
+
+  const int slot = (t < 0 ? 0 : t) % lw;
   for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
     const float2 xv = load2<T>(xn + d);
+    const float2 zv = zn ? load2<T>(zn + d) : make_float2(0.f, 0.f);
+    if (t < 0) break;  // the sequence is skipped (the same for every thread of the CTA)
     store2<T>(bx + (int64_t)slot * c + d, xv.x, xv.y);
-    if (bz) {
-      const float2 zv = zn ? load2<T>(zn + d) : make_float2(0.f, 0.f);
-      store2<T>(bz + (int64_t)slot * c + d, zv.x, zv.y);
+    if (bz) store2<T>(bz + (int64_t)slot * c + d, zv.x, zv.y);
+    if constexpr (kStaged) {
+      store2<T>(px + slot * c + d, xv.x, xv.y);
+      if (bz) store2<T>(pz + slot * c + d, zv.x, zv.y);
     }
     if (a.win) {
       const float2 v = a.apply_rope ? rope_pair(xv, pos, d, c, a.R, a.theta) : xv;
       store2<T>(static_cast<T*>(a.win) + ((int64_t)b * a.win_ring + t % a.win_ring) * c + d, v.x, v.y);
     }
   }
-  if (threadIdx.x == 0) a.buf_pos[(int64_t)b * lw + slot] = pos;
+  if (t < 0) return;
+  if (threadIdx.x == 0) bpos[slot] = pos;
+  // kStaged: the staged positions of other threads; otherwise thread 0's store above
   __syncthreads();
   if ((t + 1) % m != 0) return;
   const int w = (t + 1) / m - 1;
   if (w >= a.P_cap) return;
   const int lo = a.overlap ? (w - 1) * m : w * m;
   const int j0 = lo < 0 ? 0 : lo;
-  const int64_t epos = a.buf_pos[(int64_t)b * lw + (w * m) % lw];
+  const int eslot = (w * m) % lw;
+  const int64_t epos = eslot == slot ? pos : ppos[eslot];
   T* __restrict__ pool = static_cast<T*>(a.pool) + ((int64_t)b * a.P_cap + w) * c;
   for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
-    float2 v = pool_pair<T>(bx, bz, a.bias, lo, j0, t + 1, c, d, [lw](int j) { return (int64_t)(j % lw); });
+    float2 v = pool_pair<T>(px, pz, pb, lo, j0, t + 1, c, d, [lw](int j) { return (int64_t)(j % lw); });
     if (a.apply_rope) v = rope_pair(v, epos, d, c, a.R, a.theta);
     store2<T>(pool + d, v.x, v.y);
   }
+}
+
+// Shared memory of the staged append: Lw rows of x and z (T), of the bias (fp32) and the Lw
+// positions.
+inline size_t append_stage_bytes(const DecodeAppendArgs& a, size_t elem) {
+  const size_t lw = a.overlap ? 2 * (size_t)a.m : (size_t)a.m;
+  return lw * (size_t)a.c * (2 * elem + 4) + lw * 8;
 }
 
 cudaError_t launch_decode_append(const DecodeAppendArgs& a, int dtype, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
   int threads = ((a.c / 2 + 31) / 32) * 32;
   threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
-  if (dtype == DSV4_BF16)
-    decode_append_kernel<__nv_bfloat16><<<a.B, threads, 0, st>>>(a);
-  else
-    decode_append_kernel<float><<<a.B, threads, 0, st>>>(a);
+  const size_t elem = dtype == DSV4_BF16 ? 2 : 4;
+  const size_t stage = append_stage_bytes(a, elem);
+  const bool staged = stage <= 48 * 1024;  // within the default dynamic shared-memory limit
+  if (dtype == DSV4_BF16) {
+    if (staged)
+      decode_append_kernel<__nv_bfloat16, true><<<a.B, threads, stage, st>>>(a);
+    else
+      decode_append_kernel<__nv_bfloat16, false><<<a.B, threads, 0, st>>>(a);
+  } else {
+    if (staged)
+      decode_append_kernel<float, true><<<a.B, threads, stage, st>>>(a);
+    else
+      decode_append_kernel<float, false><<<a.B, threads, 0, st>>>(a);
+  }
   note_launch();
   return cudaGetLastError();
 }

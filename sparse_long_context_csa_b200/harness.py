@@ -95,14 +95,33 @@ def make_outputs(w, params: abi.Dsv4Params, device="cuda", scores=False) -> dict
     return o
 
 
+_SIDE_STREAMS: dict = {}
+
+
+def _side_stream(device) -> "torch.cuda.Stream":
+    if device not in _SIDE_STREAMS:
+        _SIDE_STREAMS[device] = torch.cuda.Stream(device=device)
+    return _SIDE_STREAMS[device]
+
+
 def append_token(w, params, x: dict, o: dict, k: int, stream=None) -> None:
     """Append history token k (rows x["kv"][k], x["kI"][k], ...) to every sequence's cache:
     the K=V stream (rotated window row; entry pooled and rotated when the token closes a
-    block) and the indexer-key stream (no RoPE, no window)."""
+    block) on ``stream`` and, concurrently, the indexer-key stream (no RoPE, no window) on
+    a side stream that forks from and joins back into ``stream``: the two caches share no
+    memory, and each launch is latency-bound."""
+    main = stream if stream is not None else torch.cuda.current_stream()
+    side = _side_stream(main.device)
+    fork = torch.cuda.Event()
+    fork.record(main)
+    side.wait_event(fork)
     abi.dsv4_decode_append(params, w.D, x["kv"][k], x["z"][k], x["bias"], x["pos_hist"][k], x["t_hist"][k],
-                           o["buf_x"], o["buf_z"], o["buf_pos"], 1, o["win"], o["pool"], stream=stream)
+                           o["buf_x"], o["buf_z"], o["buf_pos"], 1, o["win"], o["pool"], stream=main)
     abi.dsv4_decode_append(params, w.cI, x["kI"][k], x["zI"][k], x["biasI"], x["pos_hist"][k], x["t_hist"][k],
-                           o["bufI_x"], o["bufI_z"], o["bufI_pos"], 0, None, o["poolI"], stream=stream)
+                           o["bufI_x"], o["bufI_z"], o["bufI_pos"], 0, None, o["poolI"], stream=side)
+    join = torch.cuda.Event()
+    join.record(side)
+    main.wait_event(join)
 
 
 def append_prefill(w, params, x: dict, o: dict, stream=None) -> None:
