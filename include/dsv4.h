@@ -90,7 +90,7 @@ typedef struct dsv4_params {
  *   alpha_.[d] = softmax over J_w of (z[j,d] + bias[slot(j),d]),
  * with J_w = [(w-1)m, (w+1)m) ∩ [0,S) and slot(j) = j-(w-1)m when overlap, else
  * J_w = [wm,(w+1)m), slot(j) = j-wm.  With apply_rope, the entry's trailing R channels
- * are rotated (interleaved pairs, base rope_theta) at pos[b, w*m].
+ * are rotated (interleaved pairs, base rope_theta; R <= 128) at pos[b, w*m].
  *
  *   c      channels per row (D for the K=V stream, cI for the indexer-key stream)
  *   x      [B,S,c] T          token rows (not rotated)
@@ -128,7 +128,7 @@ dsv4_status dsv4_compress_kv(const dsv4_params* params, int32_t c, const void* x
  *   buf_x      [B,Lw,c] T          in/out: raw rows of the last Lw tokens (token j in slot j % Lw)
  *   buf_z      [B,Lw,c] T or NULL  in/out: their logits (required when z is given)
  *   buf_pos    [B,Lw] int64        in/out: their positions
- *   apply_rope rotate the window rows and the new entries (trailing R channels, rope_theta)
+ *   apply_rope rotate the window rows and the new entries (trailing R <= 128 channels, rope_theta)
  *   win        [B,win_ring,c] T or NULL  in/out: window ring; token j, rotated at its
  *                                  position when apply_rope, in slot j % win_ring
  *   pool       [B,P_cap,c] T       in/out: the pool

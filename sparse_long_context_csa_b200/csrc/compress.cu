@@ -62,17 +62,25 @@ __device__ __forceinline__ float2 pool_pair(const T* __restrict__ x, const T* __
   return make_float2(acc0 / s0, acc1 / s1);
 }
 
-// RoPE of channel pair (d, d+1) when it lies in the trailing R channels.
-__device__ __forceinline__ float2 rope_pair(float2 v, int64_t pos, int d, int c, int R, float theta) {
+// RoPE of channel pair (d, d+1) when it lies in the trailing R channels; inv_freq[k] =
+// theta^(-2k/R) comes from the host, the angle pos * inv_freq[k] is formed and reduced in
+// double precision (positions up to 2^20 keep full float accuracy in cos/sin).
+__device__ __forceinline__ float2 rope_pair(float2 v, int64_t pos, int d, int c, int R, const double* inv_freq) {
   const int rope_lo = c - R;
   if (d < rope_lo) return v;
-  float cs, sn;
-  rope_cos_sin(pos, (d - rope_lo) / 2, R, theta, &cs, &sn);
+  double sd, cd;
+  sincos((double)pos * inv_freq[(d - rope_lo) / 2], &sd, &cd);
+  const float cs = (float)cd, sn = (float)sd;
   return make_float2(v.x * cs - v.y * sn, v.x * sn + v.y * cs);
 }
 
+// theta^(-2k/R) for k < R/2 (R <= 2 * kMaxRopePairs, checked by the caller).
+inline void fill_inv_freq(double* inv, int R, float theta) {
+  for (int k = 0; k < kMaxRopePairs; ++k) inv[k] = (R > 0 && k < R / 2) ? pow((double)theta, -2.0 * k / R) : 0.0;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(256, 5) compress_kernel(CompressArgs a) {
+__global__ void __launch_bounds__(256, 5) compress_kernel(const __grid_constant__ CompressArgs a) {
   const int w = blockIdx.x;
   const int b = blockIdx.y;
   const int c = a.c;
@@ -91,7 +99,7 @@ __global__ void __launch_bounds__(256, 5) compress_kernel(CompressArgs a) {
     for (int pr = threadIdx.x; pr < c / 2; pr += blockDim.x) {
       const int d = 2 * pr;
       float2 v = pool_pair<T>(x, z, a.bias, lo, j0, hi, c, d, [](int j) { return (int64_t)j; });
-      if (a.apply_rope) v = rope_pair(v, pos[(int64_t)w * m], d, c, a.R, a.theta);
+      if (a.apply_rope) v = rope_pair(v, pos[(int64_t)w * m], d, c, a.R, a.inv_freq);
       store2<T>(pool + d, v.x, v.y);
     }
   }
@@ -103,15 +111,17 @@ __global__ void __launch_bounds__(256, 5) compress_kernel(CompressArgs a) {
     for (int it = threadIdx.x; it < (t_hi - w * m) * npairs; it += blockDim.x) {
       const int j = w * m + it / npairs;
       const int d = 2 * (it % npairs);
-      const float2 v = rope_pair(load2<T>(x + (int64_t)j * c + d), pos[j], d, c, a.R, a.theta);
+      const float2 v = rope_pair(load2<T>(x + (int64_t)j * c + d), pos[j], d, c, a.R, a.inv_freq);
       store2<T>(xr + (int64_t)j * c + d, v.x, v.y);
     }
   }
 }
 
-cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st) {
-  const int nblk = (a.S + a.m - 1) / a.m;
-  if (nblk == 0 || a.B == 0) return cudaSuccess;
+cudaError_t launch_compress(const CompressArgs& args, int dtype, cudaStream_t st) {
+  const int nblk = (args.S + args.m - 1) / args.m;
+  if (nblk == 0 || args.B == 0) return cudaSuccess;
+  CompressArgs a = args;
+  fill_inv_freq(a.inv_freq, a.R, a.theta);
   int threads = ((a.c / 2 + 31) / 32) * 32;
   threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
   dim3 grid(nblk, a.B);
@@ -136,7 +146,7 @@ cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st) {
 // (the buffered positions, written by thread 0, are read after a barrier).  Both paths pool
 // with pool_pair, so the entry has the same bits as the one the prefill compressor writes.
 template <typename T, bool kStaged>
-__global__ void __launch_bounds__(256) decode_append_kernel(DecodeAppendArgs a) {
+__global__ void __launch_bounds__(256) decode_append_kernel(const __grid_constant__ DecodeAppendArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   const int b = blockIdx.x;
   const int c = a.c, m = a.m;
@@ -187,7 +197,7 @@ __global__ void __launch_bounds__(256) decode_append_kernel(DecodeAppendArgs a) 
       if (bz) store2<T>(pz + slot * c + d, zv.x, zv.y);
     }
     if (a.win) {
-      const float2 v = a.apply_rope ? rope_pair(xv, pos, d, c, a.R, a.theta) : xv;
+      const float2 v = a.apply_rope ? rope_pair(xv, pos, d, c, a.R, a.inv_freq) : xv;
       store2<T>(static_cast<T*>(a.win) + ((int64_t)b * a.win_ring + t % a.win_ring) * c + d, v.x, v.y);
     }
   }
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(256) decode_append_kernel(DecodeAppendArgs a) 
   T* __restrict__ pool = static_cast<T*>(a.pool) + ((int64_t)b * a.P_cap + w) * c;
   for (int d = 2 * threadIdx.x; d < c; d += 2 * blockDim.x) {
     float2 v = pool_pair<T>(px, pz, pb, lo, j0, t + 1, c, d, [lw](int j) { return (int64_t)(j % lw); });
-    if (a.apply_rope) v = rope_pair(v, epos, d, c, a.R, a.theta);
+    if (a.apply_rope) v = rope_pair(v, epos, d, c, a.R, a.inv_freq);
     store2<T>(pool + d, v.x, v.y);
   }
 }
@@ -217,8 +227,10 @@ inline size_t append_stage_bytes(const DecodeAppendArgs& a, size_t elem) {
   return lw * (size_t)a.c * (2 * elem + 4) + lw * 8;
 }
 
-cudaError_t launch_decode_append(const DecodeAppendArgs& a, int dtype, cudaStream_t st) {
-  if (a.B == 0) return cudaSuccess;
+cudaError_t launch_decode_append(const DecodeAppendArgs& args, int dtype, cudaStream_t st) {
+  if (args.B == 0) return cudaSuccess;
+  DecodeAppendArgs a = args;
+  fill_inv_freq(a.inv_freq, a.R, a.theta);
   int threads = ((a.c / 2 + 31) / 32) * 32;
   threads = threads < 32 ? 32 : (threads > 256 ? 256 : threads);
   const size_t elem = dtype == DSV4_BF16 ? 2 : 4;

@@ -95,7 +95,8 @@ dsv4_status run_compress(const dsv4_params* p, int c, const void* x, const void*
   if ((z && !aligned16(z)) || (bias && !aligned16(bias)) || (x_rot && !aligned16(x_rot))) return DSV4_ERR_ALIGN;
   if (apply_rope != 0 && apply_rope != 1) return DSV4_ERR_ARG;
   if (apply_rope) {
-    if (p->R < 0 || (p->R & 1) || p->R > c || !(p->rope_theta > 0.f)) return DSV4_ERR_SHAPE;
+    if (p->R < 0 || (p->R & 1) || p->R > c || p->R > 2 * kMaxRopePairs || !(p->rope_theta > 0.f))
+      return DSV4_ERR_SHAPE;
     if (!pos) return DSV4_ERR_ARG;
     if (!aligned16(pos)) return DSV4_ERR_ALIGN;
   } else if (x_rot) {
@@ -215,7 +216,8 @@ dsv4_status dsv4_decode_append(const dsv4_params* p, int32_t c, const void* x, c
   if (z && !buf_z) return DSV4_ERR_ARG;  // logits can only be pooled from the buffer
   if (win && p->win_ring < 1) return DSV4_ERR_SHAPE;
   if (apply_rope != 0 && apply_rope != 1) return DSV4_ERR_ARG;
-  if (apply_rope && (p->R < 0 || (p->R & 1) || p->R > c || !(p->rope_theta > 0.f))) return DSV4_ERR_SHAPE;
+  if (apply_rope && (p->R < 0 || (p->R & 1) || p->R > c || p->R > 2 * kMaxRopePairs || !(p->rope_theta > 0.f)))
+    return DSV4_ERR_SHAPE;
   const void* ptrs[] = {x, z, bias, pos, t, buf_x, buf_z, buf_pos, win, pool};
   for (const void* q : ptrs)
     if (q && !aligned16(q)) return DSV4_ERR_ALIGN;

@@ -13,9 +13,13 @@ namespace dsv4 {
 // Count one kernel launch (read back by dsv4_launch_count).
 void note_launch(int n = 1);
 
+// RoPE frequencies theta^(-2k/R), k < R/2, formed on the host in double precision (R <= 128).
+constexpr int kMaxRopePairs = 64;
+
 struct CompressArgs {
   int B, S, c, m, overlap, P_cap, R, apply_rope;
   float theta;
+  double inv_freq[kMaxRopePairs];  // filled by the launcher
   const void* x;
   const void* z;
   const float* bias;
@@ -28,6 +32,7 @@ cudaError_t launch_compress(const CompressArgs& a, int dtype, cudaStream_t st);
 struct DecodeAppendArgs {
   int B, c, m, overlap, win_ring, P_cap, R, apply_rope;
   float theta;
+  double inv_freq[kMaxRopePairs];  // filled by the launcher
   const void* x;
   const void* z;
   const float* bias;

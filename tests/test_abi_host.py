@@ -141,6 +141,7 @@ def test_decode_append_rejects_bad_arguments(abi):
     assert call(_params(abi, win_ring=128), buf_z=None) == 1              # logits given but nowhere to buffer them
     assert call(_params(abi, win_ring=0)) == 2              # a window ring of no rows
     assert call(_params(abi, win_ring=128, R=63)) == 2                    # odd rope width
+    assert call(_params(abi, win_ring=128, R=130)) == 2                   # wider than the frequency table
     assert call(_params(abi, win_ring=128), apply_rope=2) == 1
     assert call(_params(abi, win_ring=128), buf_x=FAKE + 4) == 3
     assert call(_params(abi, win_ring=128, dtype=9)) == 4
@@ -156,6 +157,8 @@ def test_compress_and_layers_reject_bad_arguments(abi):
     small = _params(abi, P_cap=100)  # S/m = 2048 entries do not fit
     assert lib.dsv4_compress_kv(ctypes.byref(small), 512, FAKE, None, None, FAKE, 1, FAKE, None, None) == 2
     # sliding-window layers: no pool (P_cap 0, pool NULL) -> only the rotated rows, which are required
+    wide = _params(abi, R=130)  # RoPE frequencies are tabled for R <= 128
+    assert lib.dsv4_compress_kv(ctypes.byref(wide), 512, FAKE, None, None, FAKE, 1, FAKE, None, None) == 2
     nopool = _params(abi, P_cap=0)
     assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE, None, None, FAKE, 1, None, None, None) == 1
     assert lib.dsv4_compress_kv(ctypes.byref(nopool), 512, FAKE, None, None, FAKE, 0, None, FAKE, None) == 1
