@@ -217,7 +217,9 @@ dsv4_status dsv4_topk_select(const dsv4_params* params, const float* scores,
  *
  *   q       [B,Sq,H,D] T       rotated at qpos inside when rope_q (else already rotated)
  *   kv_win  window rows, already rotated: [B,S,D] T (win_ring == 0) or [B,win_ring,D] T
- *   pool    [B,P_cap,D] T      compressed entries, already rotated
+ *   pool    [B,P_cap,D] T      compressed entries, already rotated; NULL with P_cap == 0
+ *                              and idx NULL: a sliding-window layer ([V4] layer types,
+ *                              `sliding_attention`) attends the window alone
  *   idx     [B,Sq,topk] int32 or NULL   selected entries (-1 = empty slot); every entry
  *                              must be visible and appear once.  NULL: every visible
  *                              entry is attended (HCA, no indexer).
