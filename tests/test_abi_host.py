@@ -186,3 +186,22 @@ def test_workspace_is_a_pure_function_of_params(abi):
     assert sizes["dsa_prefill_bf16"] == 32768 * 2048 * 4 + (256 << 20)
     assert abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"])) == \
         abi.dsv4_workspace_bytes(harness.params_for(synth.WORKLOADS["tiny_csa_f32"]))
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU fallback: without the built library the binding raises instead of computing."""
+    from sparse_long_context_csa_b200 import abi as mod
+    monkeypatch.setattr(mod, "_lib", None)
+    with pytest.raises(ImportError):
+        mod.load(str(tmp_path / "libdsv4.so"))
+
+
+def test_product_package_never_imports_the_oracle():
+    """The CPU oracle is test infrastructure: nothing in the package refers to it."""
+    pkg = os.path.join(ROOT, "sparse_long_context_csa_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
+                assert "dsv4_oracle" not in src, f
