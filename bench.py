@@ -315,8 +315,10 @@ def run_reference(args, w):
     host = synth.make_inputs(w) if w.kind != "decode" else None
     per_step = []
     desc = ""
+    # each step is a bounded sample; the whole run stays within a few minutes
+    budget = min(args.ref_budget, max(1.5, 150.0 / max(1, args.warmup + args.steps)))
     for i in range(args.warmup + args.steps):
-        rate, rows, secs, desc = cpu_oracle_rate(w, args.ref_budget, host)
+        rate, rows, secs, desc = cpu_oracle_rate(w, budget, host)
         if i >= args.warmup:
             per_step.append(rate)
     if per_step_kind(w) == "us/step":
@@ -393,7 +395,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="csa_prefill_bf16", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-budget", type=float, default=12.0,
+                    help="at most this many seconds of oracle work per reference step (fewer when "
+                         "warm-up + steps would make the run longer than ~150 s)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-run", action="store_true",
