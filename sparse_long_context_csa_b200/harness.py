@@ -157,6 +157,19 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
 PARTS = ("append", "compress", "indexer_scores", "topk", "attention")
 
 
+def step_input_keys(w) -> list:
+    """The per-step activations a step reads (what a serving loop copies in every step); the
+    layer weights (compressor bias, sink) and the decode cache stay resident on the device."""
+    if w.kind == "decode":
+        return ["q", "qI", "wI", "q_index", "qpos"]
+    if w.kind == "append":
+        return ["kv", "z", "kI", "zI", "pos_hist", "t_hist"]
+    keys = ["q", "kv", "z", "pos"]
+    if w.nI > 0:
+        keys += ["qI", "wI", "kI", "zI"]
+    return keys
+
+
 def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
     """The same step as ``step`` issued entry point by entry point, the indexer as its two
     halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select): the same
