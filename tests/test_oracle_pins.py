@@ -332,6 +332,26 @@ def test_sliding_layer_equals_dense_window_attention():
     np.testing.assert_allclose(res["out"][0, 0], p[:, None] * x["kv"][0, 0][None, :16], atol=1e-12)
 
 
+def test_sliding_layer_follows_the_worked_mask():
+    """Keys of the sliding layer = the [sliding] grid of the worked 16-token example (window 8),
+    attended with the sink as an extra logit and the output rotated back by -t."""
+    g = _read_golden_sections("mask_example_16tok.txt")
+    x = _tiny_inputs(16, S=16)
+    R, theta, scale = 8, 1000.0, 0.4
+    res = O.sliding_layer(x["q"], x["kv"], x["sink"], x["pos"], n_win=8, scale=scale, dv=16, R=R, theta=theta,
+                          rotate_out=1)
+    keys = _rope_complex(x["kv"][0], x["pos"][0], R, theta)
+    for t in range(16):
+        vis = [j for j in range(16) if g["sliding"][t][j] == "1"]
+        qt = _rope_complex(x["q"][0, t], x["pos"][0, t], R, theta)
+        lg = scale * qt @ keys[vis].T
+        mx = np.maximum(lg.max(axis=1), x["sink"])
+        e = np.exp(lg - mx[:, None])
+        o = (e @ keys[vis]) / (e.sum(axis=1) + np.exp(x["sink"] - mx))[:, None]
+        np.testing.assert_allclose(res["out"][0, t], _rope_complex(o, x["pos"][0, t], R, theta, sign=-1.0),
+                                   atol=1e-12)
+
+
 def test_csa_with_topk_covering_pool_equals_dense_masked_attention():
     x = _tiny_inputs(12, S=48, m=4, overlap=1)
     kw = dict(m=4, n_win=5, scale=0.3, dv=16, R=8, theta=1000.0, rotate_out=1)
