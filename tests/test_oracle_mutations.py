@@ -58,11 +58,16 @@ MUTATIONS = [
      "            alpha = e / e.sum(axis=0)\n            entry = (alpha * x[b, js]).sum(axis=0)",
      "            alpha = e / e.sum(axis=1, keepdims=True)\n            entry = (alpha * x[b, js]).sum(axis=0)",
      [("test_compress_zero_logits_is_window_mean", {"overlap": 1}),
-      ("test_compress_gate_selects_and_slot_bias_alignment", {"overlap": 1})]),
+      ("test_compress_gate_selects_and_slot_bias_alignment", {"overlap": 1}),
+      ("test_compress_is_linear_in_the_rows_and_its_weights_sum_to_one", {})]),
     ("per-slot bias in reversed slot order",
      "logit = logit + bias[slots]", "logit = logit + bias[slots[::-1]]",
      [("test_compress_gate_selects_and_slot_bias_alignment", {"overlap": 1}),
       ("test_compress_gate_selects_and_slot_bias_alignment", {"overlap": 0})]),
+    ("sliding layer keys rotated one position late",
+     "kv_rot = store_as(rope_rotate(kv, pos, R, theta), store)\n    q_index = np.tile(np.arange(S), (B, 1))\n    out = sparse_mqa_attention(q, kv_rot, np.zeros((B, 0, D))",
+     "kv_rot = store_as(rope_rotate(kv, pos + 1, R, theta), store)\n    q_index = np.tile(np.arange(S), (B, 1))\n    out = sparse_mqa_attention(q, kv_rot, np.zeros((B, 0, D))",
+     [("test_sliding_layer_equals_dense_window_attention", {}), ("test_sliding_layer_follows_the_worked_mask", {})]),
     ("decode cache buffer slot off by one",
      'cache["raw"][t % lw] = _f64(x_t)', 'cache["raw"][(t + 1) % lw] = _f64(x_t)',
      [("test_decode_append_matches_prefill_compression", {"m": 4, "overlap": True})]),

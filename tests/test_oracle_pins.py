@@ -480,3 +480,36 @@ def test_decode_append_matches_prefill_compression(m, overlap):
     rot = O.rope_rotate(x, pos, R, 10000.0)
     for j in range(S - ring, S):
         np.testing.assert_allclose(cache["win"][j % ring], rot[0, j], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- invariants
+def test_attention_is_invariant_to_the_order_of_the_index_list():
+    """Attention is a sum over a key set: any order of the selected entries (and of the -1
+    holes among them) gives the same output."""
+    x = _tiny_inputs(17, S=40)
+    kw = dict(n_win=5, m=4, scale=0.3, dv=16, R=8, theta=1000.0, rope_q=True, rotate_out=1)
+    pool = O.compress(x["kv"], x["z"], x["bias"], x["pos"], m=4, overlap=True, apply_rope=True, R=8, theta=1000.0)
+    kv_rot = O.rope_rotate(x["kv"], x["pos"], 8, 1000.0)
+    qi = np.arange(40)[None]
+    idx = O.indexer_topk(x["qI"], x["wI"], O.compress(x["kI"], x["zI"], x["biasI"], x["pos"], m=4, overlap=True,
+                                                        apply_rope=False), qi, m=4, topk=5)
+    rng = np.random.default_rng(0)
+    shuffled = np.stack([np.stack([rng.permutation(r) for r in idx[0]])])
+    a = O.sparse_mqa_attention(x["q"], kv_rot, pool, idx, x["sink"], x["pos"], qi, **kw)
+    b = O.sparse_mqa_attention(x["q"], kv_rot, pool, shuffled, x["sink"], x["pos"], qi, **kw)
+    np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_compress_is_linear_in_the_rows_and_its_weights_sum_to_one():
+    """For fixed logits the pool is a per-channel convex combination of the window's rows:
+    linear in the rows (RoPE included), and constant rows pool to that constant."""
+    x = _tiny_inputs(18, S=32)
+    kw = dict(m=4, overlap=True, apply_rope=True, R=8, theta=1000.0)
+    y = np.random.default_rng(1).standard_normal(x["kv"].shape)
+    lhs = O.compress(2.0 * x["kv"] - 3.0 * y, x["z"], x["bias"], x["pos"], **kw)
+    rhs = 2.0 * O.compress(x["kv"], x["z"], x["bias"], x["pos"], **kw) - 3.0 * O.compress(y, x["z"], x["bias"],
+                                                                                          x["pos"], **kw)
+    np.testing.assert_allclose(lhs, rhs, atol=1e-12)
+    const = np.broadcast_to(np.linspace(-1.0, 1.0, 16), x["kv"].shape).copy()
+    pooled = O.compress(const, x["z"], x["bias"], x["pos"], m=4, overlap=True, apply_rope=False)
+    np.testing.assert_allclose(pooled, const[:, :pooled.shape[1]], atol=1e-12)  # every row is the same vector
