@@ -44,6 +44,11 @@ its status:
      are the window rows only; their RoPE base is rope_theta (10000), since
      compress_rope_theta belongs to the compressed layers.  Pinned (dense masked
      attention with an empty compressor section).
+  R14 grouped output projection: head group i = the contiguous heads [iH/g, (i+1)H/g),
+     concatenated in head order and projected by its own o_a_proj weight; the
+     groups' results, concatenated in group order, feed o_b_proj.  No biases
+     (attention_bias=False).  PARITY UNPINNED against the method (the pages give
+     the shapes only); pinned against its own closed forms.
 """
 from __future__ import annotations
 
@@ -64,6 +69,7 @@ __all__ = [
     "csa_layer",
     "hca_layer",
     "sliding_layer",
+    "grouped_out_proj",
     "new_decode_cache",
     "decode_append",
 ]
@@ -355,6 +361,27 @@ def sliding_layer(q, kv, sink, pos, *, n_win, scale, dv, R, theta, rotate_out, r
                                scale=scale, dv=dv, R=R, theta=theta, rope_q=True,
                                rotate_out=rotate_out, P_cap=0, rows=rows)
     return {"kv_rot": kv_rot, "out": out}
+
+
+# --------------------------------------------------------------------------
+# Grouped output projection  [V4] "Hybrid attention (§2.3)", grouped low-rank output
+# projection (o_a_proj, a grouped linear, then o_b_proj; o_groups, o_lora_rank).
+# --------------------------------------------------------------------------
+def grouped_out_proj(o, wa, wb):
+    """o [T,H,dv] attention outputs; wa [g, d_g, (H/g)*dv] one o_a_proj weight per head group;
+    wb [hidden, g*d_g] the o_b_proj weight.  Returns y [T, hidden] (no biases).
+
+    Reading R14: group i holds the contiguous heads [i*H/g, (i+1)*H/g); its heads' outputs,
+    concatenated in head order, are projected by its own weight to d_g channels; the g
+    results, concatenated in group order, are projected to hidden_size.
+    """
+    T, H, dv = o.shape
+    g = wa.shape[0]
+    assert H % g == 0 and wa.shape[2] == (H // g) * dv and wb.shape[1] == g * wa.shape[1]
+    hg = H // g
+    o = _f64(o)
+    u = np.concatenate([o[:, i * hg:(i + 1) * hg, :].reshape(T, hg * dv) @ _f64(wa[i]).T for i in range(g)], axis=1)
+    return u @ _f64(wb).T
 
 
 # --------------------------------------------------------------------------

@@ -68,6 +68,9 @@ MUTATIONS = [
      "kv_rot = store_as(rope_rotate(kv, pos, R, theta), store)\n    q_index = np.tile(np.arange(S), (B, 1))\n    out = sparse_mqa_attention(q, kv_rot, np.zeros((B, 0, D))",
      "kv_rot = store_as(rope_rotate(kv, pos + 1, R, theta), store)\n    q_index = np.tile(np.arange(S), (B, 1))\n    out = sparse_mqa_attention(q, kv_rot, np.zeros((B, 0, D))",
      [("test_sliding_layer_equals_dense_window_attention", {}), ("test_sliding_layer_follows_the_worked_mask", {})]),
+    ("output-projection groups interleaved instead of contiguous heads",
+     "o[:, i * hg:(i + 1) * hg, :].reshape(T, hg * dv)", "o[:, i::g, :].reshape(T, hg * dv)",
+     [("test_grouped_out_proj_equals_dense_block_diagonal_product", {}), ("test_grouped_out_proj_special_cases", {})]),
     ("decode cache buffer slot off by one",
      'cache["raw"][t % lw] = _f64(x_t)', 'cache["raw"][(t + 1) % lw] = _f64(x_t)',
      [("test_decode_append_matches_prefill_compression", {"m": 4, "overlap": True})]),

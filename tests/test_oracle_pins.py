@@ -513,3 +513,47 @@ def test_compress_is_linear_in_the_rows_and_its_weights_sum_to_one():
     const = np.broadcast_to(np.linspace(-1.0, 1.0, 16), x["kv"].shape).copy()
     pooled = O.compress(const, x["z"], x["bias"], x["pos"], m=4, overlap=True, apply_rope=False)
     np.testing.assert_allclose(pooled, const[:, :pooled.shape[1]], atol=1e-12)  # every row is the same vector
+
+
+# ---------------------------------------------------------------- grouped output projection
+def _grouped_inputs(seed, T=5, H=8, dv=6, g=4, dg=3, hidden=7):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((T, H, dv)), rng.standard_normal((g, dg, (H // g) * dv)),
+            rng.standard_normal((hidden, g * dg)))
+
+
+def test_grouped_out_proj_equals_dense_block_diagonal_product():
+    """o_a_proj as one dense product with a block-diagonal weight (block i maps the flattened
+    heads of group i to its d_g outputs), then o_b_proj: written out element by element."""
+    o, wa, wb = _grouped_inputs(0)
+    T, H, dv = o.shape
+    g, dg, width = wa.shape
+    y = O.grouped_out_proj(o, wa, wb)
+    ref = np.zeros((T, wb.shape[0]))
+    for t in range(T):
+        flat = o[t].reshape(H * dv)
+        u = np.zeros(g * dg)
+        for i in range(g):
+            for r in range(dg):
+                u[i * dg + r] = sum(wa[i, r, c] * flat[i * width + c] for c in range(width))
+        ref[t] = [sum(wb[k, j] * u[j] for j in range(g * dg)) for k in range(wb.shape[0])]
+    np.testing.assert_allclose(y, ref, atol=1e-12)
+
+
+def test_grouped_out_proj_special_cases():
+    o, wa, wb = _grouped_inputs(1)
+    T, H, dv = o.shape
+    # one group: the plain low-rank product wb @ wa @ flat(o)
+    wa1 = np.random.default_rng(2).standard_normal((1, 5, H * dv))
+    wb1 = np.random.default_rng(3).standard_normal((7, 5))
+    np.testing.assert_allclose(O.grouped_out_proj(o, wa1, wb1), o.reshape(T, -1) @ wa1[0].T @ wb1.T, atol=1e-12)
+    # identity projections give back the flattened heads
+    g = 4
+    eye_a = np.stack([np.eye((H // g) * dv)] * g)
+    np.testing.assert_allclose(O.grouped_out_proj(o, eye_a, np.eye(H * dv)), o.reshape(T, -1), atol=1e-12)
+    # heads of one group only reach that group's channels of the intermediate
+    o2 = np.zeros_like(o)
+    o2[:, 2:4] = o[:, 2:4]            # heads 2 and 3 = group 1 of 4
+    u = O.grouped_out_proj(o2, wa, np.eye(wb.shape[1]))
+    dg = wa.shape[1]
+    assert np.abs(u[:, dg:2 * dg]).max() > 0 and np.abs(np.delete(u, np.s_[dg:2 * dg], axis=1)).max() == 0
