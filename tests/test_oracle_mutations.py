@@ -78,6 +78,12 @@ MUTATIONS = [
      'entry = rope_rotate(entry, cache["pos"][(w * m) % lw], R, theta)',
      'entry = rope_rotate(entry, cache["pos"][t % lw], R, theta)',
      [("test_decode_append_matches_prefill_compression", {"m": 4, "overlap": True})]),
+    ("bf16 storage truncates instead of rounding",
+     "r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16", "r = (u >> 16).astype(np.uint32) << 16",
+     [("test_store_as_bf16_rounds_to_nearest_even", {}), ("test_store_as_matches_library_conversions", {})]),
+    ("bf16 storage rounds ties away from zero (tie-to-even term dropped)",
+     "u + 0x7FFF + ((u >> 16) & 1)", "u + 0x8000",
+     [("test_store_as_bf16_rounds_to_nearest_even", {}), ("test_store_as_matches_library_conversions", {})]),
 ]
 
 

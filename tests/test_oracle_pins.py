@@ -557,3 +557,52 @@ def test_grouped_out_proj_special_cases():
     u = O.grouped_out_proj(o2, wa, np.eye(wb.shape[1]))
     dg = wa.shape[1]
     assert np.abs(u[:, dg:2 * dg]).max() > 0 and np.abs(np.delete(u, np.s_[dg:2 * dg], axis=1)).max() == 0
+
+
+# ---------------------------------------------------------------- storage rounding
+def test_store_as_bf16_rounds_to_nearest_even():
+    """bf16 storage (7 explicit mantissa bits) of values worked out by hand: exact ties go to
+    the even neighbour (also across a binade edge and in the subnormal range), values past a
+    tie round away, signs and zeros are kept, and a float32 above the bf16 range overflows."""
+    p = 2.0 ** -8
+    cases = [
+        (1.0 + p, 1.0),                          # tie between 1 and 1 + 2^-7: even is 1
+        (1.0 + 3 * p, 1.0 + 2.0 ** -6),          # tie between 1 + 2^-7 (odd) and 1 + 2^-6 (even)
+        (-(1.0 + p), -1.0),                      # the negative tie
+        (1.0 + p + 2.0 ** -20, 1.0 + 2.0 ** -7),  # just past the tie
+        (1.0 + p - 2.0 ** -20, 1.0),             # just below it
+        (2.0 - p, 2.0),                          # tie at the top of a binade carries into the exponent
+        (2.0 - 3 * 2.0 ** -9, 2.0 - 2.0 ** -7),  # below that tie
+        (0.1, 0.10009765625),                    # 0x3DCCCCCD -> 0x3DCD
+        ((2.0 - 2.0 ** -7) * 2.0 ** 127, (2.0 - 2.0 ** -7) * 2.0 ** 127),  # largest finite bf16
+        (float(np.finfo(np.float32).max), math.inf),  # above bf16's range: rounds to infinity
+        (2.0 ** -133, 2.0 ** -133),              # smallest bf16 subnormal
+        (2.0 ** -134, 0.0),                      # tie between 0 and it: even is 0
+        (3 * 2.0 ** -134, 2.0 ** -132),          # tie between 2^-133 (odd) and 2^-132 (even)
+        (5.0, 5.0), (-7.5, -7.5),                # exactly representable values are unchanged
+    ]
+    got = O.store_as(np.array([c[0] for c in cases]), "bf16")
+    for (x, want), g in zip(cases, got):
+        assert g == want, f"store_as({x!r}, 'bf16') = {g!r}, expected {want!r}"
+    zeros = O.store_as(np.array([0.0, -0.0]), "bf16")
+    assert np.all(zeros == 0.0) and not np.signbit(zeros[0]) and np.signbit(zeros[1])
+
+
+def test_store_as_matches_library_conversions():
+    """bf16 storage equals torch's float32 -> bfloat16 conversion (round to nearest even) on a
+    grid of random values over many binades, with exact ties planted; f32 storage equals
+    numpy's float32 cast; no storage keeps float64."""
+    import torch
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(200000) * np.exp2(rng.integers(-140, 120, 200000))).astype(np.float32)
+    u = x.view(np.uint32)
+    u[::5] = (u[::5] & np.uint32(0xFFFF0000)) | np.uint32(0x8000)   # exact ties
+    u[1::5] = (u[1::5] & np.uint32(0xFFFF0000)) | np.uint32(0x7FFF)  # just below a tie
+    u[2::5] = (u[2::5] & np.uint32(0xFFFF0000)) | np.uint32(0x8001)  # just above a tie
+    x = u.view(np.float32)
+    want = torch.from_numpy(x.copy()).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.store_as(x.astype(np.float64), "bf16")
+    np.testing.assert_array_equal(got, want)
+    y = rng.standard_normal(1000) * 1e3
+    np.testing.assert_array_equal(O.store_as(y, "f32"), y.astype(np.float32).astype(np.float64))
+    np.testing.assert_array_equal(O.store_as(y, None), y)
