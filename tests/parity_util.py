@@ -30,18 +30,24 @@ def score_error_bound(qI_t, wI_t, keys, rel_key_err: float) -> np.ndarray:
     return mag * ((cI + nI + 2) * U32 + rel_key_err)
 
 
-def check_topk_row(gpu_row, scores, K, err, rel_tie=1e-6):
+def check_topk_row(gpu_row, scores, K, err, rel_tie=1e-6, stats=None):
     """Check a GPU top-k row against fp64 scores of the visible entries.
 
     Rules: the row holds min(K, vis) distinct visible entries in ascending order, then -1;
     it equals the oracle's set except for entries whose score is within the combined
     error band of the K-th score (near ties the two precisions may break differently).
     Returns the number of excused differences; raises AssertionError otherwise.
+
+    ``stats`` (a dict, optional) accumulates: rows checked, rows with a swap, swapped
+    entries, and swapped entries whose fp64 gap to the K-th score exceeds ``rel_tie``
+    relative (excused only by the fp32 accumulation band, not by the 1e-6 rule).
     """
     gpu_row = np.asarray(gpu_row)
     vis = scores.shape[0]
     n = min(K, vis)
     sel = gpu_row[:n]
+    if stats is not None:
+        stats["rows"] = stats.get("rows", 0) + 1
     assert np.all(gpu_row[n:] == -1), "slots past min(K, vis) must be -1"
     assert np.all((sel >= 0) & (sel < vis)), "selected entry not visible"
     assert np.all(np.diff(sel) > 0), "entries must be distinct and ascending"
@@ -56,10 +62,24 @@ def check_topk_row(gpu_row, scores, K, err, rel_tie=1e-6):
     band = np.maximum(err, rel_tie * abs(kth))
     extra = np.setdiff1d(sel, ref)
     missing = np.setdiff1d(ref, sel)
+    beyond = 0
     for w_ in np.concatenate([extra, missing]):
-        assert abs(scores[w_] - kth) <= band[w_] + band[order[K - 1]], (
+        gap = abs(scores[w_] - kth)
+        assert gap <= band[w_] + band[order[K - 1]], (
             f"entry {w_} differs (score {scores[w_]!r}, K-th {kth!r}, band {band[w_]!r})")
+        beyond += int(gap > rel_tie * abs(kth))
+    if stats is not None:
+        stats["rows_with_swaps"] = stats.get("rows_with_swaps", 0) + 1
+        stats["swapped_entries"] = stats.get("swapped_entries", 0) + len(extra) + len(missing)
+        stats["swaps_beyond_1e-6_rel"] = stats.get("swaps_beyond_1e-6_rel", 0) + beyond
     return len(extra)
+
+
+def report(name, stats):
+    """One line of near-tie statistics (shown with pytest -s)."""
+    print(f"[near-ties] {name}: {stats.get('rows', 0)} rows, {stats.get('rows_with_swaps', 0)} with a swap, "
+          f"{stats.get('swapped_entries', 0)} swapped entries, "
+          f"{stats.get('swaps_beyond_1e-6_rel', 0)} of them beyond 1e-6 relative")
 
 
 def assert_close_rel(got, ref, rtol, atol=0.0, what=""):
