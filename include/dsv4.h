@@ -174,6 +174,9 @@ dsv4_status dsv4_indexer_topk(const dsv4_params* params, const void* qI, const f
  *   - Every call shares the array.  Calls that overlap on the GPU (other streams, other
  *     host threads) race on it and must be serialised by the caller.  No part of the
  *     array needs to start at zero: each score row is written before it is read.
+ *   - The looked-up address is kept for the life of the process.  After cudaDeviceReset
+ *     (or anything else that destroys and recreates the device's primary context) it is
+ *     stale: do not call this entry point on that device again in the same process.
  */
 dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* params, const void* qI, const float* wI,
                                       const void* poolI, const int32_t* q_index, int32_t* idx,

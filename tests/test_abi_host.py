@@ -205,3 +205,14 @@ def test_product_package_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
                 assert "dsv4_oracle" not in src, f
+
+
+def test_noalloc_indexer_rejects_pools_beyond_its_scratch(abi):
+    """A pool of more entries than the fixed score scratch holds (4,194,304 fp32 scores) is
+    refused with DSV4_ERR_SHAPE on the host, before the scratch is looked up or any kernel is
+    enqueued: the fake addresses below are never dereferenced."""
+    lib = abi.load()
+    p = _params(abi, B=64, S=131072, Sq=1, P_cap=(4 << 20) + 1, topk=2048)
+    st = lib.dsv4_indexer_topk_noalloc(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == 2
+    # at the limit the size check passes and the call goes on to the device (not made here)
