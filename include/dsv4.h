@@ -266,6 +266,32 @@ dsv4_status dsv4_hca_layer(const dsv4_params* params, const void* q, const void*
                            const int64_t* pos, void* out, void* pool, void* kv_rot,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Grouped low-rank output projection ([V4] "Hybrid attention (§2.3)", grouped output
+ * projection: o_groups head groups -> o_lora_rank per group (DeepseekV4GroupedLinear,
+ * `o_a_proj`) -> hidden_size (`o_b_proj`); no biases).  Head group i holds the contiguous
+ * heads [i*H/g, (i+1)*H/g); their outputs, concatenated in head order, are projected by
+ * the group's own weight; the g results, concatenated in group order, feed o_b_proj:
+ *   u[t, i*dg + r] = sum_c wa[i, r, c] * o[t, i*H/g + c/dv, c % dv]     c < (H/g)*dv
+ *   y[t, k]        = sum_j wb[k, j] * u[t, j]                            j < g*dg
+ * bf16 in and out, fp32 accumulation on the tensor cores; u is rounded to bf16 between the
+ * two products.  Uses H, dv and dtype (must be DSV4_BF16) from params.
+ *
+ *   T       tokens (rows of o)
+ *   groups  o_groups (divides H);  dg  o_lora_rank (a multiple of 256)
+ *   hidden  hidden_size (a multiple of 256); (H/groups)*dv must be a multiple of 64
+ *   o       [T,H,dv] bf16      attention outputs, read in place
+ *   wa      [groups,dg,(H/groups)*dv] bf16   o_a_proj weights (one per group)
+ *   wb      [hidden,groups*dg] bf16          o_b_proj weight
+ *   u       [T,groups*dg] bf16 out: the grouped intermediate (caller-owned scratch)
+ *   y       [T,hidden] bf16    out
+ * DSV4_ERR_SHAPE for sizes the kernel does not tile (or dtype float32); validation happens
+ * on the host before any launch; allocates nothing.
+ */
+dsv4_status dsv4_grouped_out_proj(const dsv4_params* params, int32_t T, int32_t groups, int32_t dg,
+                                  int32_t hidden, const void* o, const void* wa, const void* wb, void* u,
+                                  void* y, void* stream);
+
 /* Bytes of workspace any entry point needs for these params (a pure function of them). */
 size_t dsv4_workspace_bytes(const dsv4_params* params);
 
@@ -275,10 +301,23 @@ const char* dsv4_status_string(dsv4_status status);
 /* Library ABI version (major * 100 + minor). */
 int32_t dsv4_version(void);
 
-/* Synchronise `stream`, then read and clear the device-side check word of the current
+/* Synchronise `stream`, then read and clear the device-side check words of the current
  * device: DSV4_ERR_DEVICE_CHECK means a kernel gave up a bounded pipeline wait (its CTA
- * returned early and its outputs are invalid); nothing traps or hangs instead. */
+ * returned early and its outputs are invalid), or, with dsv4_set_index_checks on, that an
+ * index list was invalid; nothing traps or hangs instead. */
 dsv4_status dsv4_device_check(void* stream);
+
+/* Device-side validation of attention index lists ([V4] "Attention mask layout": a query
+ * sees entry w only when w < (t+1)/m; empty slots hold -1; each entry is one key).  With
+ * the checks on (default: off; on in builds with DSV4_DEBUG), dsv4_sparse_mqa_attn first
+ * checks every index list it is given: an entry other than -1 that is negative or not
+ * visible sets bit 0 of a device error word, an entry that appears twice in a row sets
+ * bit 1 (rows of up to 1,572,864 visible entries; longer rows get the range check only).
+ * The attention itself still runs and never reads out of bounds (an entry that is not
+ * visible is masked).  dsv4_device_check then returns DSV4_ERR_DEVICE_CHECK and clears the
+ * word.  Nothing traps.  The switch is process-wide; it costs one extra launch per call. */
+void dsv4_set_index_checks(int32_t on);
+int32_t dsv4_index_checks(void);
 
 /* Kernels this process has enqueued through libdsv4 so far (all devices, all entry
  * points); a monotone counter for launch accounting, read without synchronising. */

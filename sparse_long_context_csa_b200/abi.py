@@ -21,7 +21,8 @@ STATUS = {0: "DSV4_OK", 1: "DSV4_ERR_ARG", 2: "DSV4_ERR_SHAPE", 3: "DSV4_ERR_ALI
 EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
             "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check", "dsv4_indexer_scores",
-            "dsv4_topk_select", "dsv4_decode_append")
+            "dsv4_topk_select", "dsv4_decode_append", "dsv4_grouped_out_proj", "dsv4_set_index_checks",
+            "dsv4_index_checks")
 
 
 class Dsv4Error(RuntimeError):
@@ -64,6 +65,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_sparse_mqa_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_csa_layer.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.dsv4_hca_layer.argtypes = [P] + [vp] * 10 + [sz, vp]
+    lib.dsv4_grouped_out_proj.argtypes = [P, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.dsv4_set_index_checks.argtypes = [i32]
+    lib.dsv4_set_index_checks.restype = None
+    lib.dsv4_index_checks.restype = i32
     lib.dsv4_workspace_bytes.argtypes = [P]
     lib.dsv4_workspace_bytes.restype = sz
     lib.dsv4_status_string.argtypes = [ctypes.c_int]
@@ -74,7 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_device_check.restype = ctypes.c_int
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
                "dsv4_hca_layer", "dsv4_indexer_topk_noalloc", "dsv4_indexer_scores", "dsv4_topk_select",
-               "dsv4_decode_append"):
+               "dsv4_decode_append", "dsv4_grouped_out_proj"):
         getattr(lib, fn).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -178,3 +183,17 @@ def dsv4_hca_layer(params, q, kv, z, bias, sink, pos, out, pool, kv_rot, workspa
     _check("dsv4_hca_layer", load().dsv4_hca_layer(
         ctypes.byref(params), _ptr(q), _ptr(kv), _ptr(z), _ptr(bias), _ptr(sink), _ptr(pos), _ptr(out),
         _ptr(pool), _ptr(kv_rot), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def dsv4_grouped_out_proj(params, T, groups, dg, hidden, o, wa, wb, u, y, stream=None):
+    _check("dsv4_grouped_out_proj",
+           load().dsv4_grouped_out_proj(ctypes.byref(params), T, groups, dg, hidden, _ptr(o), _ptr(wa), _ptr(wb),
+                                        _ptr(u), _ptr(y), _stream(stream)))
+
+
+def dsv4_set_index_checks(on: bool) -> None:
+    load().dsv4_set_index_checks(1 if on else 0)
+
+
+def dsv4_index_checks() -> bool:
+    return bool(load().dsv4_index_checks())

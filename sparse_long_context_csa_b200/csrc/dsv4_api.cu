@@ -135,6 +135,10 @@ dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, co
   a.nsplit = 1;
   const int64_t rows = (int64_t)p->B * p->Sq;
   if (rows == 0) return DSV4_OK;
+  if (idx && index_checks_on()) {
+    const cudaError_t e = launch_index_check(idx, q_index, rows, p->Sq, p->topk, p->m, p->P_cap, as_stream(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+  }
   if (attn_tc_supported(a, p->dtype)) {
     // few queries: split each query's keys over several CTAs when a workspace is given
     const size_t need = attn_split_bytes(rows, attn_keys_estimate(p), p->dv);
@@ -186,10 +190,17 @@ uint64_t dsv4_launch_count(void) { return g_launches.load(std::memory_order_rela
 
 dsv4_status dsv4_device_check(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return DSV4_ERR_CUDA;
-  int code = 0, code2 = 0;
+  int code = 0, code2 = 0, code3 = 0, code4 = 0;
   if (take_attn_tc_error(&code) != cudaSuccess) return DSV4_ERR_CUDA;
   if (take_indexer_tc_error(&code2) != cudaSuccess) return DSV4_ERR_CUDA;
-  return (code || code2) ? DSV4_ERR_DEVICE_CHECK : DSV4_OK;
+  if (take_out_proj_error(&code3) != cudaSuccess) return DSV4_ERR_CUDA;
+  if (take_index_check_error(&code4) != cudaSuccess) return DSV4_ERR_CUDA;
+  return (code || code2 || code3 || code4) ? DSV4_ERR_DEVICE_CHECK : DSV4_OK;
+}
+
+void dsv4_set_index_checks(int32_t on) { set_index_checks(on); }
+
+int32_t dsv4_index_checks(void) { return index_checks_on() ? 1 : 0;
 }
 
 size_t dsv4_workspace_bytes(const dsv4_params* p) {
@@ -367,6 +378,23 @@ dsv4_status dsv4_hca_layer(const dsv4_params* p, const void* q, const void* kv, 
   if (p->S / p->m > p->P_cap) return DSV4_ERR_SHAPE;
   if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
   return run_attn(p, q, kv_rot, pool, nullptr, sink, pos, nullptr, out, nullptr, 0, stream);
+}
+
+dsv4_status dsv4_grouped_out_proj(const dsv4_params* p, int32_t T, int32_t groups, int32_t dg, int32_t hidden,
+                                  const void* o, const void* wa, const void* wb, void* u, void* y, void* stream) {
+  if (!p) return DSV4_ERR_ARG;
+  if (p->dtype != DSV4_BF16) return p->dtype == DSV4_F32 ? DSV4_ERR_SHAPE : DSV4_ERR_DTYPE;
+  if (T < 0 || groups < 1 || dg < 1 || hidden < 1 || p->H < 1 || p->dv < 1) return DSV4_ERR_SHAPE;
+  if (p->H % groups != 0) return DSV4_ERR_SHAPE;
+  if (!o || !wa || !wb || !u || !y) return DSV4_ERR_ARG;
+  const void* ptrs[] = {o, wa, wb, u, y};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return DSV4_ERR_ALIGN;
+  OutProjArgs a{};
+  a.T = T; a.H = p->H; a.dv = p->dv; a.groups = groups; a.dg = dg; a.hidden = hidden;
+  a.o = o; a.wa = wa; a.wb = wb; a.u = u; a.y = y;
+  if (!out_proj_supported(a)) return DSV4_ERR_SHAPE;
+  return from_cuda(launch_out_proj(a, as_stream(stream)));
 }
 
 }  // extern "C"

@@ -98,4 +98,26 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
 // Read and clear the tensor-core kernel's error word (non-zero: a bounded wait gave up).
 cudaError_t take_attn_tc_error(int* code);
 
+// Grouped output projection (bf16, tensor cores): u = per-group o_a_proj of the attention
+// output, y = o_b_proj(u).
+struct OutProjArgs {
+  int T, H, dv, groups, dg, hidden;
+  const void* o;   // [T, H, dv]
+  const void* wa;  // [groups, dg, (H/groups)*dv]
+  const void* wb;  // [hidden, groups*dg]
+  void* u;         // [T, groups*dg]
+  void* y;         // [T, hidden]
+};
+bool out_proj_supported(const OutProjArgs& a);
+cudaError_t launch_out_proj(const OutProjArgs& a, cudaStream_t st);
+cudaError_t take_out_proj_error(int* code);
+
+// Optional validation of attention index lists (out of range, not visible, duplicated):
+// off by default (on in DSV4_DEBUG builds), switched by dsv4_set_index_checks.
+void set_index_checks(int on);
+bool index_checks_on();
+cudaError_t launch_index_check(const int32_t* idx, const int32_t* q_index, int64_t rows, int Sq, int topk, int m,
+                               int P_cap, cudaStream_t st);
+cudaError_t take_index_check_error(int* code);
+
 }  // namespace dsv4

@@ -8,6 +8,8 @@ A "step" is one pass of the hot path over one batch:
                      dsv4_sparse_mqa_attn over the window alone
   decode append:     dsv4_decode_append of one token per sequence to the K=V stream
                      (buffer, window ring, pool) and to the indexer-key stream
+  output projection: dsv4_grouped_out_proj of the attention output (o_a_proj per head
+                     group, then o_b_proj)
 PyTorch only allocates device memory and supplies the stream; every step of the
 method runs inside libdsv4.
 """
@@ -36,7 +38,7 @@ def torch_dtype(w):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-FLOAT_ACT = ("q", "kv", "z", "qI", "kI", "zI", "pool", "poolI", "win")  # stored in the activation dtype
+FLOAT_ACT = ("q", "kv", "z", "qI", "kI", "zI", "pool", "poolI", "win", "o", "wa", "wb")  # activation dtype
 FLOAT_F32 = ("bias", "biasI", "wI", "sink")                             # always fp32
 
 
@@ -79,6 +81,10 @@ def make_outputs(w, params: abi.Dsv4Params, device="cuda", scores=False) -> dict
     dt = torch_dtype(w)
     if w.kind == "append":
         return append_state(w, device)
+    if w.kind == "outproj":
+        T = w.B * w.Sq
+        return {"u": torch.empty((T, w.o_groups * w.o_rank), dtype=dt, device=device),
+                "out": torch.empty((T, w.hidden), dtype=dt, device=device)}
     o = {"out": torch.empty((w.B, w.Sq, w.H, w.dv), dtype=dt, device=device)}
     if w.kind != "decode":
         if w.P_cap > 0:
@@ -136,6 +142,10 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
     if w.kind == "append":
         append_token(w, params, x, o, x["kv"].shape[0] - 1, stream)
         return
+    if w.kind == "outproj":
+        abi.dsv4_grouped_out_proj(params, w.B * w.Sq, w.o_groups, w.o_rank, w.hidden, x["o"], x["wa"], x["wb"],
+                                  o["u"], o["out"], stream=stream)
+        return
     ws = o["workspace"]
     if w.kind in ("csa", "dsa"):
         abi.dsv4_csa_layer(params, x["q"], x["kv"], x.get("z"), x.get("bias"), x["qI"], x["wI"], x["kI"],
@@ -154,7 +164,7 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
         raise ValueError(w.kind)
 
 
-PARTS = ("append", "compress", "indexer_scores", "topk", "attention")
+PARTS = ("append", "compress", "indexer_scores", "topk", "attention", "out_proj")
 
 
 def step_input_keys(w) -> list:
@@ -164,6 +174,8 @@ def step_input_keys(w) -> list:
         return ["q", "qI", "wI", "q_index", "qpos"]
     if w.kind == "append":
         return ["kv", "z", "kI", "zI", "pos_hist", "t_hist"]
+    if w.kind == "outproj":
+        return ["o"]
     keys = ["q", "kv", "z", "pos"]
     if w.nI > 0:
         keys += ["qI", "wI", "kI", "zI"]
@@ -185,6 +197,11 @@ def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
         mark("append", 0)
         step(w, params, x, o, stream)
         mark("append", 1)
+        return
+    if w.kind == "outproj":
+        mark("out_proj", 0)
+        step(w, params, x, o, stream)
+        mark("out_proj", 1)
         return
     if w.kind in ("csa", "dsa", "hca", "swa"):
         mark("compress", 0)

@@ -30,6 +30,7 @@ BASE_SEED = 20261202
 STREAMS = {
     "q": 1, "kv": 2, "z": 3, "bias": 4, "qI": 5, "wI": 6, "kI": 7, "zI": 8,
     "biasI": 9, "sink": 10, "pool": 11, "poolI": 12, "win": 13, "q_index": 14,
+    "o": 16, "wa": 17, "wb": 18,
 }
 # (stream 15 draws the offsets of strided_selection)
 
@@ -38,7 +39,7 @@ STREAMS = {
 class Workload:
     name: str
     config_id: int
-    kind: str            # "csa" | "hca" | "decode" | "dsa" | "swa" (window only) | "append"
+    kind: str            # "csa" | "hca" | "decode" | "dsa" | "swa" (window only) | "append" | "outproj"
     dtype: str           # "f32" | "bf16"
     B: int
     S: int               # tokens in the sequence (prefill) / cache length (decode)
@@ -58,6 +59,9 @@ class Workload:
     P_cap: int           # pool capacity (entries per sequence)
     win_ring: int = 0    # >0: window rows live in a ring of this many slots
     qindex_spread: int = 0
+    o_groups: int = 0    # grouped output projection: head groups, o_lora_rank, hidden_size
+    o_rank: int = 0
+    hidden: int = 0
 
     @property
     def scale(self) -> float:
@@ -99,6 +103,11 @@ WORKLOADS = {
                                        Sq=1, H=64, D=512, R=64, dv=512, n_win=128, m=4, overlap=1,
                                        nI=8, cI=128, topk=2048, theta=160000.0, rotate_out=1,
                                        P_cap=32768, win_ring=128, qindex_spread=1024),
+    # the grouped output projection of the CSA prefill's attention output (8192 tokens, 64
+    # heads x 512): o_groups 8, o_lora_rank 1024, hidden_size 4096 (DeepseekV4Config defaults)
+    "out_proj_bf16": Workload("out_proj_bf16", 7, "outproj", "bf16", B=1, S=8192, Sq=8192, H=64, D=512,
+                              R=0, dv=512, n_win=0, m=1, overlap=0, nI=0, cI=0, topk=0, theta=10000.0,
+                              rotate_out=0, P_cap=0, o_groups=8, o_rank=1024, hidden=4096),
 }
 
 
@@ -193,6 +202,13 @@ def tensor_specs(w: Workload, gains: dict | None = None) -> dict:
                 "kI": spec("kI", (lw * w.B, w.cI), 1 / math.sqrt(w.cI)),
                 "zI": spec("zI", (lw * w.B, w.cI), 1.0),
                 "biasI": spec("biasI", (lw, w.cI), 0.1, bf16=False)}
+    if w.kind == "outproj":
+        # attention outputs (one value row's scale) and the two projection weights, each
+        # N(0,1)/sqrt(fan_in)
+        width = (w.H // w.o_groups) * w.dv
+        return {"o": spec("o", (w.B * w.Sq, w.H, w.dv), 1 / math.sqrt(w.dv)),
+                "wa": spec("wa", (w.o_groups * w.o_rank, width), 1 / math.sqrt(width)),
+                "wb": spec("wb", (w.hidden, w.o_groups * w.o_rank), 1 / math.sqrt(w.o_groups * w.o_rank))}
     specs = {
         "q": spec("q", (w.B * w.Sq, w.H, w.D), 1 / math.sqrt(w.D)),
         "sink": spec("sink", (w.H,), 1.0, bf16=False),
@@ -246,7 +262,8 @@ def reshape(w: Workload, name: str, a: np.ndarray) -> np.ndarray:
         "q": (w.B, w.Sq, w.H, w.D), "kv": (w.B, w.S, w.D), "z": (w.B, w.S, w.D),
         "qI": (w.B, w.Sq, w.nI, w.cI), "wI": (w.B, w.Sq, w.nI), "kI": (w.B, w.S, w.cI),
         "zI": (w.B, w.S, w.cI), "pool": (w.B, w.P_cap, w.D), "poolI": (w.B, w.P_cap, w.cI),
-        "win": (w.B, w.win_ring, w.D),
+        "win": (w.B, w.win_ring, w.D), "o": (w.B * w.Sq, w.H, w.dv),
+        "wa": (w.o_groups, w.o_rank, (w.H // w.o_groups) * w.dv if w.o_groups else 0),
     }
     return a.reshape(shapes[name]) if name in shapes else a
 
@@ -261,7 +278,7 @@ def make_inputs(w: Workload, gains: dict | None = None, threads: int = 8) -> dic
         t = out["q_index"][:, 0][None, :] - np.arange(lw - 1, -1, -1, dtype=np.int64)[:, None]
         out["t_hist"] = t.astype(np.int32)
         out["pos_hist"] = t.astype(np.int64)
-    elif w.kind != "decode":
+    elif w.kind not in ("decode", "outproj"):
         out["pos"] = token_positions(w)
     return out
 

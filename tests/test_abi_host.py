@@ -216,3 +216,27 @@ def test_noalloc_indexer_rejects_pools_beyond_its_scratch(abi):
     st = lib.dsv4_indexer_topk_noalloc(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None)
     assert st == 2
     # at the limit the size check passes and the call goes on to the device (not made here)
+
+
+def test_grouped_out_proj_rejects_untiled_sizes_on_the_host(abi):
+    """Sizes the tensor-core tiles do not cover, float32 activations, null or misaligned
+    pointers are refused before any CUDA call (fake addresses, never dereferenced)."""
+    import synth
+    from sparse_long_context_csa_b200 import harness
+    lib = abi.load()
+    w = synth.WORKLOADS["out_proj_bf16"]
+    p = harness.params_for(w)
+    ok = dict(T=16, groups=8, dg=256, hidden=512)
+    cases = [(dict(dg=200), 2), (dict(hidden=300), 2), (dict(groups=3), 2), (dict(T=-1), 2)]
+    for bad, want in cases:
+        kw = {**ok, **bad}
+        st = lib.dsv4_grouped_out_proj(ctypes.byref(p), kw["T"], kw["groups"], kw["dg"], kw["hidden"],
+                                       FAKE, FAKE, FAKE, FAKE, FAKE, None)
+        assert st == want, (bad, st)
+    st = lib.dsv4_grouped_out_proj(ctypes.byref(p), 16, 8, 256, 512, FAKE, FAKE, None, FAKE, FAKE, None)
+    assert st == 1
+    st = lib.dsv4_grouped_out_proj(ctypes.byref(p), 16, 8, 256, 512, FAKE + 8, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == 3
+    p32 = harness.params_for(w.replace(dtype="f32"))
+    st = lib.dsv4_grouped_out_proj(ctypes.byref(p32), 16, 8, 256, 512, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == 2

@@ -61,7 +61,7 @@ def test_units_and_l2_policy_of_every_workload():
     # inputs larger than L2 need no flush; the append's few rows and the tiny case do
     assert flush == {"tiny_csa_f32": True, "csa_prefill_bf16": False, "hca_prefill_bf16": False,
                      "csa_decode_bf16": False, "dsa_prefill_bf16": False, "swa_prefill_bf16": False,
-                     "csa_decode_append_bf16": True}
+                     "csa_decode_append_bf16": True, "out_proj_bf16": False}
     for n, w in synth.WORKLOADS.items():
         c = bench.config_of(w)
         assert c["workload"] == n and ("flushed" in c["l2"]) == flush[n]
