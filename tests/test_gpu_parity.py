@@ -425,3 +425,45 @@ def test_bench_step_path_swa_prefill(lib):
     g = _np(o["out"])
     for b, s in rows:
         assert_max_abs(g[b, s], ref["out"][b, s], ATTN_TOL["bf16"], f"window-only row {s}")
+
+
+def test_index_checks_report_bad_lists(lib):
+    """With the index checks on, dsv4_sparse_mqa_attn validates its index lists on the device:
+    a valid list passes; a duplicated entry, an entry that is not yet visible and an entry
+    below -1 each make dsv4_device_check report DSV4_ERR_DEVICE_CHECK (the attention still
+    runs, masking what it cannot use, and nothing traps)."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_prefill_bf16"].replace(S=1024, Sq=1024, P_cap=256, topk=64)
+    c = _cache(w)
+    x = _query_inputs(w)
+    idx = synth.strided_selection(w, x["q_index"])
+    params = harness.params_for(w)
+    d = harness.to_device(w, {"q": x["q"], "win": c["win"], "pool": c["pool"], "sink": x["sink"],
+                              "qpos": x["qpos"], "q_index": x["q_index"]})
+    out = torch.empty((w.B, w.Sq, w.H, w.dv), dtype=torch.bfloat16, device="cuda")
+
+    def run(lists):
+        abi.dsv4_sparse_mqa_attn(params, d["q"], d["win"], d["pool"], torch.from_numpy(lists).cuda(), d["sink"],
+                                 d["qpos"], d["q_index"], out)
+
+    abi.dsv4_device_check()  # start from a clear word
+    abi.dsv4_set_index_checks(True)
+    try:
+        assert abi.dsv4_index_checks()
+        run(idx)
+        abi.dsv4_device_check()
+        t = 900                       # vis = 225 entries, 64 selected
+        vis = (t + 1) // w.m
+        for name, edit in (("duplicate", lambda r: r.__setitem__(1, r[0])),
+                           ("not visible", lambda r: r.__setitem__(0, vis)),
+                           ("below -1", lambda r: r.__setitem__(2, -5))):
+            bad = idx.copy()
+            edit(bad[0, t])
+            run(bad)
+            with pytest.raises(abi.Dsv4Error) as e:
+                abi.dsv4_device_check()
+            assert e.value.status == 6, name
+            abi.dsv4_device_check()   # the word was cleared by the failing check
+    finally:
+        abi.dsv4_set_index_checks(False)
+    assert not abi.dsv4_index_checks()
