@@ -73,8 +73,17 @@ def part_work(w, q_index):
     append: bytes per sequence and stream of c channels: the new row and its logits read and
       written to the buffer (+ its position), the rotated window row (K=V stream); when the
       token closes a block, the Lw buffered rows and logits read and the entry written.
+    out_proj: 2 T (H dv dg + g dg hidden) FLOPs (the g group products, then o_b_proj); bytes =
+      o, both weights, the bf16 intermediate written and read back, and y.
     """
     e = 2 if w.dtype == "bf16" else 4
+    if w.kind == "outproj":
+        T = w.B * w.Sq
+        inner = w.o_groups * w.o_rank
+        flops = 2.0 * T * (w.H * w.dv * w.o_rank + inner * w.hidden)
+        nbytes = e * (T * w.H * w.dv + inner * (w.H // w.o_groups) * w.dv + w.hidden * inner
+                      + 2 * T * inner + T * w.hidden)
+        return {"out_proj": (flops, nbytes)}
     if w.kind == "append":
         lw = 2 * w.m if w.overlap else w.m
         t = q_index.reshape(-1).astype(np.int64)
@@ -105,18 +114,33 @@ def part_work(w, q_index):
     return work
 
 
-def roofline_of(name, flops, nbytes, ms, peaks, peak_src):
+def tensor_peak_kind(timed_ms: float, clocks: dict) -> str:
+    """Which measured bf16 peak a tensor-bound kernel is held to: the burst figure when the
+    timed region is short (under a second) or the sampled SM clock stayed at its maximum,
+    the sustained (power-capped) figure for a long region that ran below the maximum clock."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if timed_ms < 1000.0 or (sm and mx and sm >= 0.97 * mx):
+        return "burst"
+    return "sustained"
+
+
+def roofline_of(name, flops, nbytes, ms, peaks, peak_src, kind="burst"):
     """Roofline entry of one kernel: bound = the larger of its tensor time and HBM time at
-    the measured peaks; achieved = its algorithmic work / its CUDA-event time."""
-    pk_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    the measured peaks; achieved = its algorithmic work / its CUDA-event time.  A tensor
+    bound is held to the burst or the sustained bf16 peak (``kind``); the other fraction is
+    reported beside it."""
+    pk_burst = peaks["bf16_tflops"]
+    pk_sus = peaks.get("bf16_tflops_sustained", pk_burst)
+    pk_t = pk_burst if kind == "burst" else pk_sus
     pk_b = peaks["hbm_gbs"]
     t_tensor = flops / (pk_t * 1e12)
     t_hbm = nbytes / (pk_b * 1e9)
     if t_tensor >= t_hbm:
         ach = flops / (ms / 1e3) / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": pk_t, "unit": "TFLOP/s", "frac": ach / pk_t,
+                "frac_of_burst": ach / pk_burst, "frac_of_sustained": ach / pk_sus,
                 "kernel": name, "kernel_ms": ms, "algorithmic_flops": flops,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+                "peak_source": f"{peak_src} bf16_tflops ({kind})"}
     ach = nbytes / (ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": ach, "peak": pk_b, "unit": "GB/s", "frac": ach / pk_b,
             "kernel": name, "kernel_ms": ms, "algorithmic_bytes": nbytes, "peak_source": f"{peak_src} hbm_gbs"}
@@ -244,6 +268,15 @@ def cpu_oracle_rate(w, budget_s: float, host=None):
                 break
         dt = time.perf_counter() - t0
         return done / dt, done, dt, f"{done} of {w.B} decode sequences (indexer + top-k + attention)"
+    if w.kind == "outproj":
+        # blocks of 16 tokens through both projections until the budget is spent
+        done = 0
+        T = w.B * w.Sq
+        while done < T and time.perf_counter() - t0 < budget_s:
+            O.grouped_out_proj(host["o"][done:done + 16], host["wa"], host["wb"])
+            done = min(T, done + 16)
+        dt = time.perf_counter() - t0
+        return done / dt, done, dt, f"{done} of {T} tokens through o_a_proj (8 groups) and o_b_proj"
     if w.kind == "append":
         # per sequence: the Lw-1 earlier tokens are appended untimed, the step's token timed
         lw = host["kv"].shape[0]
@@ -365,6 +398,8 @@ def l2_flush_needed(w) -> bool:
     """True when a step's inputs fit in the 126 MB L2: such steps are timed with L2 flushed."""
     if w.kind == "append":
         return True
+    if w.kind == "outproj":
+        return w.B * w.Sq * w.H * w.dv * 2 <= (126 << 20)
     if w.kind == "decode":
         return w.B * w.P_cap * (w.D + w.cI) * 2 <= (126 << 20)
     return w.B * w.Sq * w.H * w.D * 2 <= (126 << 20)
@@ -379,6 +414,9 @@ def config_of(w):
         c = {"workload": w.name, "B": w.B, "cache_tokens": w.S, "head_dim": w.D, "rope_dim": w.R, "m": w.m,
              "overlap": w.overlap, "buffer_rows": 2 * w.m if w.overlap else w.m, "window_ring": w.win_ring,
              "pool_cap": w.P_cap, "index_head_dim": w.cI}
+    if w.kind == "outproj":
+        c = {"workload": w.name, "tokens": w.B * w.Sq, "H": w.H, "dv": w.dv, "o_groups": w.o_groups,
+             "o_lora_rank": w.o_rank, "hidden_size": w.hidden}
     if l2_flush_needed(w):
         c["l2"] = "L2 flushed between steps (a 256 MiB buffer written outside the timed events)"
     elif w.kind == "decode":
@@ -388,13 +426,192 @@ def config_of(w):
     return c
 
 
+EXTRA_WORKLOADS = ("hca_prefill_bf16", "csa_decode_bf16", "dsa_prefill_bf16", "out_proj_bf16")
+
+
+class Runner:
+    """One rank's device state for timing workloads (the process group, if any, is set up)."""
+
+    def __init__(self, args, world, rank, local):
+        import torch
+        from sparse_long_context_csa_b200 import abi, harness
+        self.torch, self.abi, self.harness = torch, abi, harness
+        self.args, self.world, self.rank, self.local = args, world, rank, local
+        self.sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                                    else local)
+        if not args.profile_run:
+            self.sampler.start()
+        abi.load()
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(self, v: float) -> float:
+        return reduce_max(v, self.world, "cuda")
+
+    def device_check(self, what: str):
+        """Every bounded wait in the kernels must have ended in time: a CTA that gave one up
+        returned early with invalid output, so its step must not count as a timed step."""
+        try:
+            self.abi.dsv4_device_check()
+        except self.abi.Dsv4Error as e:
+            raise SystemExit(f"bench: device-side check failed after {what}: {e}")
+
+    def setup(self, w):
+        torch, harness = self.torch, self.harness
+        host = synth.make_inputs(w)
+        params = harness.params_for(w)
+        x = harness.to_device(w, host)
+        o = harness.make_outputs(w, params, scores=True)
+        return {"w": w, "host": host, "params": params, "x": x, "o": o, "stream": torch.cuda.current_stream()}
+
+    def measure(self, st, steps: int, warmup: int):
+        """W untimed warm-up steps, then K timed steps (CUDA events on the launching stream,
+        every part bracketed by its own events); returns the max-over-ranks times."""
+        torch, harness, abi = self.torch, self.harness, self.abi
+        w, params, x, o, stream = st["w"], st["params"], st["x"], st["o"], st["stream"]
+        q_index = st["host"]["q_index"]
+        parts = [p for p in harness.PARTS if p in part_work(w, q_index)]
+
+        def step(events=None):
+            harness.step_parts(w, params, x, o, stream, events=events)
+
+        if w.kind == "append":
+            harness.append_prefill(w, params, x, o, stream)  # the cache just before the step's token
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if l2_flush_needed(w) else None
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        t_w = time.time()
+        while not self.args.profile_run and time.time() - t_w < 1.0:  # the clock sampler settles
+            step()
+            torch.cuda.synchronize()
+        self.device_check(f"the warm-up of {w.name}")
+        evs = [{p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for p in parts}
+               for _ in range(steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)] if flush is not None else None
+        self.barrier()
+        torch.cuda.synchronize()
+        n0 = abi.dsv4_launch_count()
+        wall0 = time.time()
+        start.record(stream)
+        for i in range(steps):
+            if flush is not None:
+                flush.fill_(i & 255)  # evicts the previous step's lines from L2; not inside the step's events
+                step_ev[i][0].record(stream)
+            step(evs[i])
+            if flush is not None:
+                step_ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        wall1 = time.time()
+        n1 = abi.dsv4_launch_count()
+        self.device_check(f"the timed steps of {w.name}")
+        self.barrier()
+        total_ms = start.elapsed_time(end) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
+        ms = self.max_over_ranks(total_ms)
+        part_ms = {p: self.max_over_ranks(float(np.mean([e[p][0].elapsed_time(e[p][1]) for e in evs])))
+                   for p in parts}
+        return {"ms": ms, "part_ms": part_ms, "parts": parts, "launches": int(n1 - n0),
+                "clocks": self.sampler.summary(wall0, wall1)}
+
+    def roofline(self, w, q_index, m):
+        peaks, peak_src = _peaks()
+        work = part_work(w, q_index)
+        parts, part_ms = m["parts"], m["part_ms"]
+        kind = tensor_peak_kind(m["ms"], m["clocks"])
+        dom = max(parts, key=lambda p: part_ms[p])
+        roof = roofline_of(dom, work[dom][0], work[dom][1], part_ms[dom], peaks, peak_src, kind)
+        roof["traffic"] = ncu_traffic(w.name, dom)
+        roof["parts_ms"] = part_ms
+        roof["others"] = {p: {k: v for k, v in roofline_of(p, work[p][0], work[p][1], part_ms[p], peaks, peak_src,
+                                                           kind).items()
+                              if k in ("bound", "achieved", "unit", "frac")} for p in parts if p != dom}
+        return roof
+
+    def e2e(self, st, steps: int):
+        """The same metric through the layer entry point: every step copies its activations in
+        from pinned host memory and its output back.  Steps are pipelined over two buffer sets:
+        step i's inputs go in on one copy stream while step i-1 computes and its output goes
+        out on a second copy stream (the decode append, whose result is cache state, runs
+        serially).  Returns (ms per step, h2d bytes, d2h bytes)."""
+        torch, harness = self.torch, self.harness
+        w, params, x, o, stream, host = st["w"], st["params"], st["x"], st["o"], st["stream"], st["host"]
+        keys = [k for k in harness.step_input_keys(w) if k in x]
+        host_t = harness.to_device(w, {k: host[k] for k in keys}, device=None, pin=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if w.kind == "append":
+            last = host["kv"].shape[0] - 1
+            pairs = [(x[k][last], host_t[k][last]) for k in keys]
+            result = o["buf_pos"]   # the buffer's position record (the rows stay on the device)
+            out_host = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
+            h2d = sum(t.numel() * t.element_size() for _, t in pairs)
+            d2h = out_host.numel() * out_host.element_size()
+
+            def e2e_run(n):
+                for _ in range(n):
+                    for dst, src in pairs:
+                        dst.copy_(src, non_blocking=True)
+                    harness.step(w, params, x, o, stream)
+                    out_host.copy_(result, non_blocking=True)
+
+            e2e_run(1)
+            torch.cuda.synchronize()
+            self.barrier()
+            e0.record(stream)
+            e2e_run(steps)
+            e1.record(stream)
+        else:
+            sets = [x, {**x, **{k: torch.empty_like(x[k]) for k in keys}}]
+            outs = [o, {**o, "out": torch.empty_like(o["out"])}]
+            out_host = [torch.empty(o["out"].shape, dtype=o["out"].dtype, pin_memory=True) for _ in range(2)]
+            h2d = sum(host_t[k].numel() * host_t[k].element_size() for k in keys)
+            d2h = out_host[0].numel() * out_host[0].element_size()
+            s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+            in_ready, in_free, out_ready, out_free = ([torch.cuda.Event() for _ in range(2)] for _ in range(4))
+
+            def e2e_run(n):
+                for i in range(n):
+                    b = i % 2
+                    s_in.wait_event(in_free[b])        # the step two back has read this input set
+                    with torch.cuda.stream(s_in):
+                        for k in keys:
+                            sets[b][k].copy_(host_t[k], non_blocking=True)
+                    in_ready[b].record(s_in)
+                    stream.wait_event(in_ready[b])
+                    stream.wait_event(out_free[b])     # this output buffer has been copied out
+                    harness.step(w, params, sets[b], outs[b], stream)
+                    in_free[b].record(stream)
+                    out_ready[b].record(stream)
+                    s_out.wait_event(out_ready[b])
+                    with torch.cuda.stream(s_out):
+                        out_host[b].copy_(outs[b]["out"], non_blocking=True)
+                    out_free[b].record(s_out)
+
+            e2e_run(2)
+            torch.cuda.synchronize()
+            self.barrier()
+            e0.record(s_in)
+            e2e_run(steps)
+            e1.record(s_out)
+        torch.cuda.synchronize()
+        self.device_check(f"the end-to-end steps of {w.name}")
+        return self.max_over_ranks(e0.elapsed_time(e1)) / steps, h2d, d2h
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="csa_prefill_bf16", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(synth.WORKLOADS),
+                    help="time this workload alone (default: CSA prefill as the headline, then the "
+                         "HCA prefill, CSA decode and DSA prefill workloads under \"workloads\")")
     ap.add_argument("--ref-budget", type=float, default=12.0,
                     help="at most this many seconds of oracle work per reference step (fewer when "
                          "warm-up + steps would make the run longer than ~150 s)")
@@ -403,13 +620,13 @@ def main():
     ap.add_argument("--profile-run", action="store_true",
                     help="for profilers: only the warm-up and timed steps (no clock sampler, e2e or cpu_baseline)")
     args = ap.parse_args()
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[args.workload or "csa_prefill_bf16"]
+    extras = [] if (args.workload or args.profile_run) else list(EXTRA_WORKLOADS)
     if args.impl == "reference":
         return run_reference(args, w)
 
     import torch
     import torch.distributed as dist
-    from sparse_long_context_csa_b200 import abi, harness
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -419,164 +636,49 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        return reduce_max(v, world, "cuda")
-
-    abi.load()
-    host = synth.make_inputs(w)
-    params = harness.params_for(w)
-    x = harness.to_device(w, host)
-    o = harness.make_outputs(w, params, scores=True)
-    stream = torch.cuda.current_stream()
-    q_index = host["q_index"]
-    parts = [p for p in harness.PARTS if p in part_work(w, q_index)]
-
-    def step(events=None):
-        harness.step_parts(w, params, x, o, stream, events=events)
-
-    if w.kind == "append":
-        harness.append_prefill(w, params, x, o, stream)  # the cache just before the step's token
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if l2_flush_needed(w) else None
-
-    # warm-up (also starts the clock sampler and lets it settle)
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
-    if not args.profile_run:
-        sampler.start()
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    t_w = time.time()
-    while not args.profile_run and time.time() - t_w < 1.0:  # keep the GPU busy while nvidia-smi starts
-        step()
-        torch.cuda.synchronize()
-
-    # timed region: K steps, device time; every part bracketed by its own events
-    evs = [{p: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for p in parts}
-           for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)] if flush is not None else None
-    barrier()
-    torch.cuda.synchronize()
-    n0 = abi.dsv4_launch_count()
-    wall0 = time.time()
-    start.record(stream)
-    for i in range(args.steps):
-        if flush is not None:
-            flush.fill_(i & 255)  # evicts the previous step's lines from L2; not inside the step's events
-            step_ev[i][0].record(stream)
-        step(evs[i])
-        if flush is not None:
-            step_ev[i][1].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize()
-    wall1 = time.time()
-    n1 = abi.dsv4_launch_count()
-    barrier()
-    total_ms = start.elapsed_time(end) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
-    ms = max_over_ranks(total_ms)
-    part_ms = {p: max_over_ranks(float(np.mean([e[p][0].elapsed_time(e[p][1]) for e in evs]))) for p in parts}
-    clocks = sampler.summary(wall0, wall1)
+    run = Runner(args, world, rank, local)
+    st = run.setup(w)
+    m = run.measure(st, args.steps, args.warmup)
+    ms = m["ms"]
     if args.profile_run:
         if rank == 0:
-            print(json.dumps({"profile_run": True, "ms_per_step": ms / args.steps, "part_ms": part_ms}), flush=True)
+            print(json.dumps({"profile_run": True, "ms_per_step": ms / args.steps, "part_ms": m["part_ms"]}),
+                  flush=True)
         return
 
-    # end to end through the layer entry point: every step copies its activations in from
-    # pinned host memory and its output back.  Steps are pipelined over two buffer sets: step
-    # i's inputs go in on one copy stream while step i-1 computes and its output goes out on
-    # a second copy stream (the decode append, whose result is cache state, runs serially).
-    keys = [k for k in harness.step_input_keys(w) if k in x]
-    host_t = harness.to_device(w, {k: host[k] for k in keys}, device=None, pin=True)
-    e2e_steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if w.kind == "append":
-        last = host["kv"].shape[0] - 1
-        pairs = [(x[k][last], host_t[k][last]) for k in keys]
-        result = o["buf_pos"]   # the buffer's position record (the rows stay on the device)
-        out_host = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for _, t in pairs)
-        d2h = out_host.numel() * out_host.element_size()
-
-        def e2e_run(n):
-            for _ in range(n):
-                for dst, src in pairs:
-                    dst.copy_(src, non_blocking=True)
-                harness.step(w, params, x, o, stream)
-                out_host.copy_(result, non_blocking=True)
-
-        e2e_run(1)
-        torch.cuda.synchronize()
-        barrier()
-        e0.record(stream)
-        e2e_run(e2e_steps)
-        e1.record(stream)
-    else:
-        sets = [x, {**x, **{k: torch.empty_like(x[k]) for k in keys}}]
-        outs = [o, {**o, "out": torch.empty_like(o["out"])}]
-        out_host = [torch.empty(o["out"].shape, dtype=o["out"].dtype, pin_memory=True) for _ in range(2)]
-        h2d = sum(host_t[k].numel() * host_t[k].element_size() for k in keys)
-        d2h = out_host[0].numel() * out_host[0].element_size()
-        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        in_ready, in_free, out_ready, out_free = ([torch.cuda.Event() for _ in range(2)] for _ in range(4))
-
-        def e2e_run(n):
-            for i in range(n):
-                b = i % 2
-                s_in.wait_event(in_free[b])        # the step two back has read this input set
-                with torch.cuda.stream(s_in):
-                    for k in keys:
-                        sets[b][k].copy_(host_t[k], non_blocking=True)
-                in_ready[b].record(s_in)
-                stream.wait_event(in_ready[b])
-                stream.wait_event(out_free[b])     # this output buffer has been copied out
-                harness.step(w, params, sets[b], outs[b], stream)
-                in_free[b].record(stream)
-                out_ready[b].record(stream)
-                s_out.wait_event(out_ready[b])
-                with torch.cuda.stream(s_out):
-                    out_host[b].copy_(outs[b]["out"], non_blocking=True)
-                out_free[b].record(s_out)
-
-        e2e_run(2)
-        torch.cuda.synchronize()
-        barrier()
-        e0.record(s_in)
-        e2e_run(e2e_steps)
-        e1.record(s_out)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    sampler.stop()
-
+    e2e_ms, h2d, d2h = run.e2e(st, max(3, min(args.steps, 10)))
     tokens = w.B * w.Sq
-    ms_step = ms / args.steps
     value, unit, hib = job_value(w.kind, world, tokens, args.steps, ms)
     e2e_val = job_value(w.kind, world, tokens, 1, e2e_ms)[0]
-
-    peaks, peak_src = _peaks()
-    work = part_work(w, q_index)
-    dom = max(parts, key=lambda p: part_ms[p])
-    roof = roofline_of(dom, work[dom][0], work[dom][1], part_ms[dom], peaks, peak_src)
-    roof["traffic"] = ncu_traffic(w.name, dom)
-    roof["parts_ms"] = part_ms
-    roof["others"] = {p: {k: v for k, v in roofline_of(p, work[p][0], work[p][1], part_ms[p], peaks, peak_src).items()
-                          if k in ("bound", "achieved", "unit", "frac")} for p in parts if p != dom}
-
+    roof = run.roofline(w, st["host"]["q_index"], m)
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": hib, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": hib, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1)/sqrt(d) inputs, no weights)",
             "config": config_of(w), "parallelism": f"replicas x{world} (independent sequences)",
-            "gpu_launches": int(n1 - n0), "clocks": clocks, "roofline": roof,
+            "gpu_launches": m["launches"], "clocks": m["clocks"], "roofline": roof,
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, rows, secs, desc = cpu_oracle_rate(w, args.cpu_budget, host)
+        rate, rows, secs, desc = cpu_oracle_rate(w, args.cpu_budget, st["host"])
         cv = (1e6 / rate * w.B) if per_step_kind(w) == "us/step" else rate
         line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": blas_threads(), "kind": "oracle",
                                 "sample": desc, "seconds": round(secs, 2)}
+    del st
+    # the other configurations the metric names, each its own timed region on the same rank(s)
+    others = {}
+    for name in extras:
+        wx = synth.WORKLOADS[name]
+        torch.cuda.empty_cache()
+        sx = run.setup(wx)
+        k = max(3, min(args.steps, 10))
+        mx = run.measure(sx, k, max(3, min(args.warmup, 5)))
+        vx, ux, hx = job_value(wx.kind, world, wx.B * wx.Sq, k, mx["ms"])
+        others[name] = {"value": vx, "unit": ux, "higher_is_better": hx, "steps": k,
+                        "ms_per_step": mx["ms"] / k, "gpu_launches": mx["launches"], "clocks": mx["clocks"],
+                        "config": config_of(wx), "roofline": run.roofline(wx, sx["host"]["q_index"], mx)}
+        del sx
+    if others:
+        line["workloads"] = others
+    run.sampler.stop()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
