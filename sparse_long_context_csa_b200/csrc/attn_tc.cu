@@ -15,8 +15,10 @@
 //    handing the previous tile's probabilities to the MMA: the copies overlap PV.  (Measured
 //    on B200: random 128-byte row pieces move at ~18 B/clk per SM from 2 issuing warps and
 //    ~55 B/clk from 8; TMA tile::gather4 ran at ~7 B/clk, and 128-row TMA boxes of window
-//    rows were slower than cp.async as well.)  Every chunk has its own full/free barrier
-//    pair, so S^T starts on the first chunk that lands.
+//    rows were slower than cp.async as well.)  Every chunk has its own "full" barrier, so
+//    S^T starts on the first chunk that lands; the whole tile is released by one barrier
+//    committed after its PV products (a tcgen05.commit between MMA groups holds up the
+//    issuing thread, so PV is issued as one uninterrupted run of MMAs).
 //  * Scores are computed transposed, S^T[key, head] = K_tile . Q^T (M = 128 keys keeps the
 //    tensor core at full rate; 64 heads alone would be a half-rate M=64 shape), and the same
 //    shared-memory tile is read again as V^T (MN-major) for O^T[dim, head] += V^T . P^T: K=V
@@ -93,8 +95,9 @@ struct QDesc {
 };
 
 struct Misc {
-  uint64_t cfull[kMaxChunks], cfree[kMaxChunks];
-  uint64_t qfull, qready, qfree, odone, sfull, pfull;
+  uint64_t cfull[kMaxChunks];
+  uint64_t qfull, qready, qfree, sfull, pfull;
+  uint64_t odone;  // PV of a tile done: O^T is current and the key tile may be overwritten
   uint64_t dfull[2], dfree[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -117,8 +120,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const AttnArgs& a = P.a;
   const int D = a.D;
   const int nch = D / 64;
-  const bool alias = D > 512;
-  const int nvch = a.dv / 64;  // chunks that are also value channels
   const int nvt = a.dv / 128;
   const Smem L = smem_layout(D);
   Misc* ms = reinterpret_cast<Misc*>(smem + L.misc);
@@ -133,7 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int c = 0; c < kMaxChunks; ++c) {
       tc::mbar_init(&ms->cfull[c], 256);  // one cp.async arrival per softmax thread
-      tc::mbar_init(&ms->cfree[c], 1);
     }
     tc::mbar_init(&ms->qfull, 1);
     tc::mbar_init(&ms->qready, 32);
@@ -313,8 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (lane == 0) {
           tc::umma_commit(&ms->sfull);
-          for (int c = nvch; c < nch; ++c)
-            if (!(alias && c == nch - 1)) tc::umma_commit(&ms->cfree[c]);
           if (i == ntiles - 1) tc::umma_commit(&ms->qfree);
         }
         __syncwarp();
@@ -333,10 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
                 tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
               }
-              tc::umma_commit(&ms->cfree[2 * j]);
-              tc::umma_commit(&ms->cfree[2 * j + 1]);
             }
-            if (alias) tc::umma_commit(&ms->cfree[nch - 1]);
             tc::umma_commit(&ms->odone);
           }
           __syncwarp();
@@ -393,8 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           src[j] = win_base + (int64_t)(a.win_ring ? jj % a.win_ring : jj) * D + cu * 8;
         }
       }
+      if (gcopy > 0 && !wait_ok(&ms->odone, (gcopy - 1) & 1)) ms->abort_flag = 1;
       for (int c = 0; c < nch; ++c) {
-        if (gcopy > 0 && !wait_ok(&ms->cfree[c], (gcopy - 1) & 1)) ms->abort_flag = 1;
         uint8_t* cb = smem + L.k + c * 16384;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
