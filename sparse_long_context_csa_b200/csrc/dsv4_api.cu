@@ -68,7 +68,17 @@ size_t scores_bytes(const dsv4_params* p) {
   if (rows == 0 || p->P_cap == 0 || p->nI < 1 || p->topk < 1) return 0;  // no indexer
   int64_t r = indexer_rows_per_chunk(rows, p->P_cap, kScoresBudget);
   if (r < 1) r = 1;
-  return (size_t)r * p->P_cap * sizeof(float);
+  size_t bytes = (size_t)r * p->P_cap * sizeof(float);
+  // one query per sequence (decode): the fused scores + top-k kernel keeps each split's
+  // candidates in the same space
+  IndexerArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.nI = p->nI; a.cI = p->cI; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk;
+  a.q_index = reinterpret_cast<const int32_t*>(16);  // decode plans use cache indices; never read
+  if (p->Sq == 1 && indexer_tc_supported(a, p->dtype)) {
+    const size_t sel = indexer_tc_select_bytes(a, r);
+    if (sel > bytes) bytes = sel;
+  }
+  return bytes;
 }
 
 // idx kept in the workspace by dsv4_csa_layer (a prefill call: Sq == S).
@@ -115,6 +125,7 @@ dsv4_status run_indexer(const dsv4_params* p, const void* qI, const float* wI, c
   a.B = p->B; a.Sq = p->Sq; a.nI = p->nI; a.cI = p->cI; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk;
   a.qI = qI; a.wI = wI; a.poolI = poolI; a.q_index = q_index; a.idx = idx;
   a.scores = static_cast<float*>(scores);
+  a.scores_cap = scores_cap;
   const int64_t rows = (int64_t)p->B * p->Sq;
   a.rows_per_chunk = indexer_rows_per_chunk(rows, p->P_cap, scores_cap < kScoresBudget ? scores_cap : kScoresBudget);
   if (rows == 0) return DSV4_OK;

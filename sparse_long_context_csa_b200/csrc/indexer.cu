@@ -392,6 +392,12 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st
   const int64_t rows = (int64_t)a.B * a.Sq;
   for (int64_t r0 = 0; r0 < rows; r0 += a.rows_per_chunk) {
     const int64_t r1 = r0 + a.rows_per_chunk < rows ? r0 + a.rows_per_chunk : rows;
+    if (indexer_tc_supported(a, dtype)) {
+      // one query per sequence (decode): scores and top-k in one kernel when it applies
+      const cudaError_t f = launch_indexer_tc_select(a, r0, r1, a.scores_cap, st);
+      if (f == cudaSuccess) continue;
+      if (f != cudaErrorNotSupported) return f;
+    }
     cudaError_t e = launch_indexer_scores(a, dtype, r0, r1, st);
     if (e != cudaSuccess) return e;
     e = launch_topk(a, r0, r1, st);

@@ -22,6 +22,15 @@
 // generic per-column loop issued ~6x the instructions and held the kernel at 4% of the
 // tensor pipe).  Tiles past the largest visible entry count of the group are skipped
 // (causality).  Grid: (entry splits, query groups).
+//
+// Fused top-k (one query per sequence, decode; "DeepSeek-V3.2" doc, DSA item 2: the indices
+// go straight to the attention).  The scores of a CTA's split stay in shared memory; after
+// scoring, all 16 warps select the split's top-k candidates there (select.cuh), write them
+// (order key << 32 | entry) to the work space, and count the split done on a per-query
+// counter.  The CTA that counts last merges every split's candidates (keys copied once into
+// the free stage buffers) into the query's index row, in ascending entry order.  No CTA waits
+// for another, the score rows never reach memory, and the separate top-k launch is gone.  Its
+// split of the pool comes from a cost model that also counts the selection and the merge.
 #include <cuda.h>
 #include <cstddef>
 #include <cstdint>
@@ -30,6 +39,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 #include "tc_ptx.cuh"
 
 namespace dsv4 {
@@ -52,19 +62,27 @@ struct IdxTcParams {
   int QB;                  // queries per group
   int Npad;                // QB * nI rounded up to 16
   int tiles_per_split;     // entry tiles per CTA along grid.x
+  // fused selection (one query per group): scores stay in shared memory, each CTA keeps its
+  // split's top-k candidates (order key << 32 | entry) and the last CTA of a sequence merges
+  int select;
+  int cand_stride;         // candidates kept per split: min(topk, entries per split)
+  uint64_t* cand;          // [rows, gridDim.x, cand_stride] candidates of each split
+  int* done;               // [rows] splits finished (zero before the launch; reset by the merge)
 };
 
 struct IdxSmem {
-  uint32_t a, b, misc, total;
+  uint32_t a, b, misc, sel, total;
 };
 
-__host__ __device__ inline IdxSmem idx_smem_layout(int cI, int Npad) {
+// sel_entries: scores kept in shared memory by the fused selection (0: none)
+__host__ __device__ inline IdxSmem idx_smem_layout(int cI, int Npad, int sel_entries = 0) {
   IdxSmem s;
   const int nch = cI / 64;
   s.a = 0;                                          // kStages x nch x 16 KB
   s.b = s.a + kStages * nch * 16384;                // nch x Npad x 128 B
   s.misc = s.b + nch * ((Npad * 128 + 1023) / 1024) * 1024;
-  s.total = s.misc + 4096;
+  s.sel = s.misc + 4096;                            // sel_entries fp32 scores
+  s.total = s.sel + (uint32_t)sel_entries * 4;
   return s;
 }
 
@@ -73,6 +91,7 @@ struct IdxMisc {
   uint32_t tmem_base;
   int maxvis;
   int abort_flag;
+  int sel_last;  // fused selection: this CTA merges the splits of its query
   int vis[256];
   alignas(16) float w[256 + 32];  // (query, head) weights, read as float4; zero past the group
 };
@@ -131,14 +150,23 @@ __device__ __forceinline__ void score_tile(uint32_t taddr, int k_lo, int k_hi, c
   }
 }
 
+constexpr int kSelThreads = 512;           // threads of the fused selection (all 16 warps)
+constexpr int kSelMaxEntries = 16384;      // scores per CTA kept for it (64 KB)
+constexpr int kSelKeysOffset = 20480;      // merge: candidate keys after the histogram and shared words
+constexpr int64_t kSelMinEntries = int64_t(1) << 20;  // scored entries per launch below which it is not used
+
+__device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 3, 512;" ::: "memory"); }
+
+template <bool kSelect>
 __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const IndexerArgs& a = P.a;
   const int cI = a.cI, nI = a.nI, QB = P.QB, Npad = P.Npad;
   const int lg_nI = 31 - __clz(nI);
   const int nch = cI / 64;
-  const IdxSmem L = idx_smem_layout(cI, Npad);
+  const IdxSmem L = idx_smem_layout(cI, Npad, kSelect ? P.tiles_per_split * kTileE : 0);
   IdxMisc* ms = reinterpret_cast<IdxMisc*>(smem + L.misc);
+  float* ssc = reinterpret_cast<float*>(smem + L.sel);  // fused selection: this CTA's scores
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((tc::smem_u32(smem) & 1023u) != 0) {
     if (tid == 0) atomicExch(&g_indexer_tc_error, 3);
@@ -188,6 +216,11 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
   const int t_lo = blockIdx.x * P.tiles_per_split;
   const int t_hi = min(ntile_all, t_lo + P.tiles_per_split);
   const int ntiles = t_hi > t_lo ? t_hi - t_lo : 0;
+  if (kSelect && ntile_all == 0 && blockIdx.x == 0) {
+    // nothing visible yet: the whole row is -1
+    int32_t* out = a.idx + rbase * (int64_t)a.topk;
+    for (int i = tid; i < a.topk; i += kThreads) out[i] = -1;
+  }
   if (ntiles == 0) return;
   if (warp == 4) {
     tc::tmem_alloc(&ms->tmem_base, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
@@ -276,6 +309,8 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
       }
       __syncwarp();
     }
+  } else if (warp >= 13) {
+    // fused selection launches: three more warps that only join the selection
   } else {
     // ---------------------------------------------------------------- epilogue (8 warps)
     const int q4 = warp & 3;
@@ -314,7 +349,10 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
             float sc = 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) sc = fmaf(qcol[j] == q ? wsm[j] : 0.f, fmaxf(acc[j], 0.f), sc);
-            if (w < ms->vis[q]) a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
+            if (kSelect)
+              ssc[i * kTileE + e] = sc;  // one query per group; entries past vis are never read
+            else if (w < ms->vis[q])
+              a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
           }
         }
       } else {
@@ -340,6 +378,78 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 2 * Npad <= 32 ? 32 : (2 * Npad <= 64 ? 64 : (2 * Npad <= 128 ? 128 : (2 * Npad <= 256 ? 256 : 512))));
   }
+  if constexpr (kSelect) {
+    if (tid >= kSelThreads) return;
+    // ------------------------------------------------------------ split top-k (warps 0-7)
+    // The pipeline's stage buffers are free now: they hold the radix histogram and the
+    // selection's shared words.
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.a);
+    SelShared<kSelThreads>* sh = reinterpret_cast<SelShared<kSelThreads>*>(smem + L.a + kSelBins * 4);
+    const int K = a.topk;
+    const int vis = ms->vis[0];
+    const int per = P.tiles_per_split * kTileE;  // entries per split
+    const int w0 = t_lo * kTileE;
+    const int n_loc = min(ntiles * kTileE, vis - w0);
+    const int stride = P.cand_stride;
+    uint64_t* cand = P.cand + ((int64_t)(rbase - P.row0) * gridDim.x + blockIdx.x) * stride;
+    if (n_loc <= K) {
+      for (int i = tid; i < n_loc; i += kSelThreads)
+        cand[i] = ((uint64_t)order_key(ssc[i]) << 32) | (uint32_t)(w0 + i);
+    } else {
+      select_topk<kSelThreads>(
+          n_loc, K, tid, [&](int i) { return order_key(ssc[i]); },
+          [&](int slot, int i) { cand[slot] = ((uint64_t)order_key(ssc[i]) << 32) | (uint32_t)(w0 + i); }, hist, sh,
+          sel_sync);
+    }
+    // the last split of this query to finish merges (no CTA waits for another)
+    __threadfence();
+    sel_sync();
+    const int nonempty = (ntile_all + P.tiles_per_split - 1) / P.tiles_per_split;
+    if (tid == 0) ms->sel_last = atomicAdd(&P.done[rbase - P.row0], 1) == nonempty - 1;
+    sel_sync();
+    if (!ms->sel_last) return;
+    __threadfence();
+    // the candidates of all splits in split order (ascending entries): every split but the
+    // last holds `stride` of them, the last min(topk, its visible entries); read through L2
+    const uint64_t* all = P.cand + (int64_t)(rbase - P.row0) * gridDim.x * stride;
+    const int full = (nonempty - 1) * stride;
+    const int n_tot = full + min(K, vis - (nonempty - 1) * per);
+    auto cand_at = [&](int i) {
+      const int sp = i < full ? i / stride : nonempty - 1;
+      return __ldcg(all + (int64_t)sp * stride + (i - sp * stride));
+    };
+    int32_t* out = a.idx + rbase * (int64_t)K;
+    if (n_tot <= K) {
+      for (int i = tid; i < K; i += kSelThreads) out[i] = i < n_tot ? (int32_t)(uint32_t)cand_at(i) : -1;
+    } else {
+      // the candidates' keys go to shared memory once (after the histogram and the shared
+      // words, in the free stage buffers); the radix passes then read them from there
+      uint32_t* mk = reinterpret_cast<uint32_t*>(smem + L.a + kSelKeysOffset);
+      for (int sp = 0; sp < nonempty; ++sp) {
+        const int nc = sp < nonempty - 1 ? stride : n_tot - full;
+        const uint64_t* src = all + (int64_t)sp * stride;
+        uint32_t* dst = mk + sp * stride;
+        for (int i0 = 0; i0 < nc; i0 += 8 * kSelThreads) {  // eight loads in flight per thread
+          uint64_t v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            v[u] = i < nc ? __ldcg(src + i) : 0ull;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            if (i < nc) dst[i] = (uint32_t)(v[u] >> 32);
+          }
+        }
+      }
+      sel_sync();
+      select_topk<kSelThreads>(
+          n_tot, K, tid, [&](int i) { return mk[i]; },
+          [&](int slot, int i) { out[slot] = (int32_t)(uint32_t)cand_at(i); }, hist, sh, sel_sync);
+    }
+    if (tid == 0) P.done[rbase - P.row0] = 0;  // ready for the next launch
+  }
 }
 
 }  // namespace
@@ -362,7 +472,10 @@ int indexer_num_sms() {
   return n;
 }
 
-cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+// Launch plan of the tensor-core indexer over rows [r0, r1) on nsm SMs; max_tps caps the entry
+// tiles per CTA (0: no cap).
+static IdxTcParams plan_indexer_tc(const IndexerArgs& a, int64_t r0, int64_t r1, int max_tps, int nsm,
+                                   dim3* grid_out, bool select = false) {
   IdxTcParams P{};
   P.a = a;
   P.row0 = r0;
@@ -385,11 +498,26 @@ cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r
   // (measured: 320 CTAs in 2.2 waves held the decode indexer to 63% of HBM bandwidth).
   // Prefill (no cache indices) is causal: tile counts grow along the groups and are known
   // here, so the same cost is evaluated over the CTAs that have work.
-  const int nsm = indexer_num_sms();
   int best_tps = max_tiles;
-  if (a.q_index) {
+  const int tps_hi = max_tps > 0 && max_tps < max_tiles ? max_tps : max_tiles;
+  if (a.q_index && select) {
+    // fused selection, in units of one scored tile (measured on B200, decode shapes): a split
+    // selects over its entries at ~1/4 tile per tile it scored, and the last split of a query
+    // merges every split's min(topk, entries) candidates at ~1/400 tile per candidate
+    double best_cost = 1e300;
+    for (int tps = tps_hi; tps >= 1; --tps) {
+      const int ns = (max_tiles + tps - 1) / tps;
+      const int64_t waves = (ngroups * ns + nsm - 1) / nsm;
+      const int stride = a.topk < tps * kTileE ? a.topk : tps * kTileE;
+      const double cost = waves * (1.25 * tps + 2.0) + (ns > 1 ? 0.0026 * ns * stride : 0.0);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best_tps = tps;
+      }
+    }
+  } else if (a.q_index) {
     int64_t best_cost = INT64_MAX;
-    for (int tps = max_tiles; tps >= 1; --tps) {
+    for (int tps = tps_hi; tps >= 1; --tps) {
       const int ns = (max_tiles + tps - 1) / tps;
       const int64_t waves = (ngroups * ns + nsm - 1) / nsm;
       const int64_t cost = waves * (tps + 2);
@@ -410,7 +538,7 @@ cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r
       ++groups_with[(mv + kTileE - 1) / kTileE];
     }
     int64_t best_cost = INT64_MAX;
-    for (int tps = max_tiles; tps >= 1; --tps) {
+    for (int tps = tps_hi; tps >= 1; --tps) {
       int64_t n = 0;
       for (int k = 1; k <= max_tiles; ++k) n += groups_with[k] * ((k + tps - 1) / tps);
       const int64_t cost = ((n + nsm - 1) / nsm) * (tps + 2);
@@ -420,14 +548,69 @@ cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r
       }
     }
   }
+  if (max_tps > 0 && best_tps > max_tps) best_tps = max_tps;
   P.tiles_per_split = best_tps;
   const int nsplit = (max_tiles + best_tps - 1) / best_tps;
+  *grid_out = dim3((unsigned)nsplit, (unsigned)ngroups);
+  return P;
+}
 
+cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st) {
+  dim3 grid;
+  const IdxTcParams P = plan_indexer_tc(a, r0, r1, 0, indexer_num_sms(), &grid);
   const IdxSmem L = idx_smem_layout(a.cI, P.Npad);
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  cudaError_t e =
+      cudaFuncSetAttribute(indexer_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)nsplit, (unsigned)ngroups);
-  indexer_tc_kernel<<<grid, kThreads, L.total, st>>>(P);
+  indexer_tc_kernel<false><<<grid, kThreads, L.total, st>>>(P);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// Fused scores + top-k for one query per sequence (decode): split top-k in each CTA, merged by
+// the last CTA of each query.  Work space (a.scores, ws_bytes): the per-query split counters,
+// then the candidates.  Returns cudaErrorNotSupported when the shapes or the work space do
+// not allow it (the caller then runs the two kernels).
+// (planned for the 148 SMs of a B200, so that the size is a function of the sizes alone; on
+// another SM count the plan may need more and the two-kernel path runs instead)
+size_t indexer_tc_select_bytes(const IndexerArgs& a, int64_t rows) {
+  if (a.Sq != 1 || a.nI > 16 || rows < 1) return 0;
+  dim3 grid;
+  const IdxTcParams P = plan_indexer_tc(a, 0, rows, kSelMaxEntries / kTileE, 148, &grid, true);
+  const int per = P.tiles_per_split * kTileE;
+  const size_t stride = (size_t)(a.topk < per ? a.topk : per);
+  return ((size_t)rows * sizeof(int) + 255) / 256 * 256 + (size_t)rows * grid.x * stride * sizeof(uint64_t);
+}
+
+cudaError_t launch_indexer_tc_select(const IndexerArgs& a, int64_t r0, int64_t r1, size_t ws_bytes,
+                                     cudaStream_t st) {
+  if (a.Sq != 1 || a.nI > 16 || !a.idx) return cudaErrorNotSupported;
+  // Measured on B200: the fused kernel is ahead from about a million scored entries per launch
+  // (64 queries x 32768 entries: 144 us against 152 us for the two kernels), behind below it
+  // (32 x 15000: 67 against 60 us), where too few splits leave SMs idle.
+  if ((r1 - r0) * (int64_t)a.P_cap < kSelMinEntries) return cudaErrorNotSupported;
+  dim3 grid;
+  IdxTcParams P = plan_indexer_tc(a, r0, r1, kSelMaxEntries / kTileE, indexer_num_sms(), &grid, true);
+  if (P.QB != 1) return cudaErrorNotSupported;
+  const int64_t rows = r1 - r0;
+  const int nsplit = (int)grid.x;
+  const int per = P.tiles_per_split * kTileE;
+  P.cand_stride = a.topk < per ? a.topk : per;
+  // the merge keeps every split's candidate keys in the stage buffers
+  const int64_t merge_keys = (int64_t)nsplit * P.cand_stride;
+  if (merge_keys * 4 > (int64_t)kStages * (a.cI / 64) * 16384 - kSelKeysOffset) return cudaErrorNotSupported;
+  const size_t done_bytes = ((size_t)rows * sizeof(int) + 255) / 256 * 256;
+  const size_t need = done_bytes + (size_t)rows * nsplit * P.cand_stride * sizeof(uint64_t);
+  if (need > ws_bytes) return cudaErrorNotSupported;
+  P.select = 1;
+  P.done = reinterpret_cast<int*>(a.scores);
+  P.cand = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(a.scores) + done_bytes);
+  const IdxSmem L = idx_smem_layout(a.cI, P.Npad, P.tiles_per_split * kTileE);
+  cudaError_t e = cudaMemsetAsync(P.done, 0, (size_t)rows * sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(indexer_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  if (e != cudaSuccess) return e;
+  indexer_tc_kernel<true><<<grid, kSelThreads, L.total, st>>>(P);
   note_launch();
   return cudaGetLastError();
 }
@@ -445,3 +628,4 @@ cudaError_t take_indexer_tc_error(int* code) {
 }
 
 }  // namespace dsv4
+

@@ -55,6 +55,7 @@ struct IndexerArgs {
   int32_t* idx;
   float* scores;        // workspace: [rows_per_chunk, P_cap] fp32
   int64_t rows_per_chunk;
+  size_t scores_cap;    // bytes at `scores` (the fused decode path keeps its candidates there)
 };
 cudaError_t launch_indexer_topk(const IndexerArgs& a, int dtype, cudaStream_t st);
 // The two halves of launch_indexer_topk for query rows [r0, r1): score row r lives at
@@ -64,6 +65,13 @@ cudaError_t launch_topk(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream
 // Tensor-core score kernel (bf16): scores of rows [r0, r1) into a.scores.
 bool indexer_tc_supported(const IndexerArgs& a, int dtype);
 cudaError_t launch_indexer_tc_scores(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream_t st);
+// Fused scores + top-k for one query per sequence (decode); a.scores is ws_bytes of work space.
+// cudaErrorNotSupported when the shapes or the work space do not allow it.
+cudaError_t launch_indexer_tc_select(const IndexerArgs& a, int64_t r0, int64_t r1, size_t ws_bytes,
+                                     cudaStream_t st);
+// Work space the fused path needs for `rows` queries of one query per sequence (0: the path
+// does not apply to these shapes).
+size_t indexer_tc_select_bytes(const IndexerArgs& a, int64_t rows);
 cudaError_t take_indexer_tc_error(int* code);
 // Rows of queries whose scores fit in `bytes` of score workspace.
 int64_t indexer_rows_per_chunk(int64_t total_rows, int P_cap, size_t bytes);

@@ -164,7 +164,7 @@ def step(w, params, x: dict, o: dict, stream=None) -> None:
         raise ValueError(w.kind)
 
 
-PARTS = ("append", "compress", "indexer_scores", "topk", "attention", "out_proj")
+PARTS = ("append", "compress", "indexer_topk", "indexer_scores", "topk", "attention", "out_proj")
 
 
 def step_input_keys(w) -> list:
@@ -183,9 +183,10 @@ def step_input_keys(w) -> list:
 
 
 def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
-    """The same step as ``step`` issued entry point by entry point, the indexer as its two
-    halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select): the same
-    kernels on the same data.  ``events`` maps names of ``PARTS`` to (start, end) CUDA
+    """The same step as ``step`` issued entry point by entry point: for prefill the indexer as
+    its two halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select), the same
+    kernels on the same data; for decode dsv4_indexer_topk, whose one kernel scores and
+    selects.  ``events`` maps names of ``PARTS`` to (start, end) CUDA
     event pairs recorded on ``stream`` around that part."""
     ws = o.get("workspace")
 
@@ -211,9 +212,14 @@ def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
             abi.dsv4_compress_kv(params, w.cI, x["kI"], x.get("zI"), x.get("biasI"), None, 0, o["poolI"], None,
                                  stream=stream)
         mark("compress", 1)
-    if w.nI > 0:
-        poolI = o["poolI"] if w.kind != "decode" else x["poolI"]
-        q_index = x["q_index"] if w.kind == "decode" else None
+    if w.kind == "decode":
+        # one query per sequence: dsv4_indexer_topk scores and selects in one kernel
+        mark("indexer_topk", 0)
+        abi.dsv4_indexer_topk(params, x["qI"], x["wI"], x["poolI"], x["q_index"], o["idx"], ws, stream=stream)
+        mark("indexer_topk", 1)
+    elif w.nI > 0:
+        poolI = o["poolI"]
+        q_index = None
         mark("indexer_scores", 0)
         abi.dsv4_indexer_scores(params, x["qI"], x["wI"], poolI, q_index, o["scores"], stream=stream)
         mark("indexer_scores", 1)

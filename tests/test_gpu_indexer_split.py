@@ -122,3 +122,37 @@ def test_split_calls_equal_fused_call(lib, name):
     abi.dsv4_indexer_topk(params, d["qI"], d["wI"], d["poolI"], d["q_index"], idx_b, ws)
     abi.dsv4_device_check()
     assert torch.equal(idx_a, idx_b)
+
+
+@pytest.mark.parametrize("B,S,P_cap,topk,spread", [(64, 131072, 32768, 2048, 1024), (48, 100000, 24576, 2048, 99990),
+                                                    (128, 40000, 10000, 512, 39990)])
+def test_fused_decode_indexer_matches_the_two_kernel_path(lib, B, S, P_cap, topk, spread):
+    """One query per sequence (decode) at a million scored entries or more: dsv4_indexer_topk
+    scores and selects in one kernel (split top-k in each CTA, merged by the last CTA of each
+    query).  Its index lists must equal, bit for bit, those of the two separate kernels
+    (dsv4_indexer_scores, then dsv4_topk_select) on the same inputs.  Three queries are moved
+    to the start of their caches (no visible entry, or one); the wider spreads put more below
+    topk visible entries."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, S=S, P_cap=P_cap, topk=topk, qindex_spread=spread)
+    sp = synth.cache_specs(w)
+    specs = synth.tensor_specs(w)
+    qi, _ = synth.positions(w)
+    qi[:3, 0] = [0, 2, 3]  # two queries with no visible entry yet, one with a single entry
+    host = {"qI": synth.reshape(w, "qI", specs["qI"].full()), "wI": synth.reshape(w, "wI", specs["wI"].full()),
+            "poolI": sp["poolI"].full().reshape(w.B, w.P_cap, w.cI), "q_index": qi}
+    p = harness.params_for(w)
+    d = harness.to_device(w, host)
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(p), 256), dtype=torch.uint8, device="cuda")
+    fused = torch.full((w.B, 1, w.topk), -7, dtype=torch.int32, device="cuda")
+    for _ in range(2):  # twice: the per-query split counters must be left ready for the next call
+        abi.dsv4_indexer_topk(p, d["qI"], d["wI"], d["poolI"], d["q_index"], fused, ws)
+    scores = torch.empty((w.B, w.P_cap), dtype=torch.float32, device="cuda")
+    split = torch.full((w.B, 1, w.topk), -7, dtype=torch.int32, device="cuda")
+    abi.dsv4_indexer_scores(p, d["qI"], d["wI"], d["poolI"], d["q_index"], scores)
+    abi.dsv4_topk_select(p, scores, d["q_index"], split)
+    abi.dsv4_device_check()
+    assert torch.equal(fused, split)
+    vis = np.minimum((qi[:, 0] + 1) // w.m, w.P_cap)
+    kept = (fused.cpu().numpy()[:, 0] >= 0).sum(axis=1)
+    np.testing.assert_array_equal(kept, np.minimum(vis, w.topk))
