@@ -67,6 +67,8 @@ def part_work(w, q_index):
       the gathered rows of its one query).
     indexer_scores: visible entries x nI x cI x 2 FLOPs; bytes = the indexer pool once per
       sequence + qI + wI + the fp32 score rows written.
+    indexer_topk (decode: scores and selection in one kernel): the same FLOPs; bytes = the
+      indexer pool once per sequence + qI + wI + the index rows written.
     topk: no FLOPs; bytes = the fp32 score rows read + the index rows written.
     compress: bytes = token rows (kv and kI) and their logits (m > 1) read, pools and the
       rotated K=V rows written.
@@ -104,9 +106,14 @@ def part_work(w, q_index):
                           nq * w.H * (w.D + w.dv) * e + kv_bytes + (nq * w.topk * 4 if w.topk else 0))}
     if w.nI > 0:
         pool_once = float(w.B) * float(vis.reshape(w.B, -1).max(axis=1).mean()) * w.cI * e
-        work["indexer_scores"] = (vis.sum() * w.nI * w.cI * 2.0,
-                                  pool_once + nq * w.nI * (w.cI * e + 4) + vis.sum() * 4)
-        work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
+        if w.kind == "decode":
+            # one kernel: the indexer pool once, qI and wI in, the index rows out
+            work["indexer_topk"] = (vis.sum() * w.nI * w.cI * 2.0,
+                                    pool_once + nq * w.nI * (w.cI * e + 4) + nq * w.topk * 4)
+        else:
+            work["indexer_scores"] = (vis.sum() * w.nI * w.cI * 2.0,
+                                      pool_once + nq * w.nI * (w.cI * e + 4) + vis.sum() * 4)
+            work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
     if w.kind != "decode":
         ch = w.D + (w.cI if w.nI else 0)
         rows_in = w.B * w.S * ch * e * (2 if w.m > 1 else 1)
@@ -155,10 +162,10 @@ _ATTN_SOURCE = (("attn_tc.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.
                 ("internal.h", None))
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
-    # window 128): dram__bytes_read.sum 564.3 MB + dram__bytes_write.sum 494.1 MB.  (Re-keyed
-    # when internal.h gained the RoPE frequency tables of the compressor's argument structs;
-    # nothing the attention kernel compiles changed.)
-    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "15a551fd5e1c31b13d109116e012491d251522424102b7a6bdc9cda9e60d0687", 1058375936),
+    # window 128): dram__bytes_read.sum 564.5 MB + dram__bytes_write.sum 494.9 MB.  (Re-keyed
+    # when internal.h gained the declarations of the fused decode indexer; nothing the attention
+    # kernel compiles changed.)
+    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "b3cb36a671c61b983f22101489a6f62d82dd55cdd1e046e506c8f8a88a8516a8", 1059356928),
 }
 
 
