@@ -160,12 +160,21 @@ def roofline_of(name, flops, nbytes, ms, peaks, peak_src, kind="burst"):
 # null until the kernel is captured again.  Values: (source segments, sha256, bytes per launch).
 _ATTN_SOURCE = (("attn_tc.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("common.cuh", None),
                 ("internal.h", None))
+_INDEXER_SOURCE = (("indexer_tc.cu", "\n}  // namespace\n\nbool indexer_tc_supported"), ("tc_ptx.cuh", None),
+                   ("common.cuh", None), ("internal.h", None), ("select.cuh", None))
+_OUT_PROJ_SOURCE = (("out_proj.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("internal.h", None))
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
     # window 128): dram__bytes_read.sum 564.5 MB + dram__bytes_write.sum 494.9 MB.  (Re-keyed
     # when internal.h gained the declarations of the fused decode indexer; nothing the attention
     # kernel compiles changed.)
     ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "b3cb36a671c61b983f22101489a6f62d82dd55cdd1e046e506c8f8a88a8516a8", 1059356928),
+    # ncu --set full, one launch of the CSA decode step (64 queries, pool 32768, top-2048): the fused
+    # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.5 MB.
+    ("csa_decode_bf16", "indexer_topk"): (_INDEXER_SOURCE, "228d6bc7b952cb7e18ac0173d08a4c71bd602164a3e3e02af47dcdba5dc1df87", 539299328),
+    # ncu --set full, both launches of one output-projection step (o_a_proj, then o_b_proj; the
+    # part is the two launches): 608.2 + 117.7 + 604.0 + 61.5 MB.
+    ("out_proj_bf16", "out_proj"): (_OUT_PROJ_SOURCE, "272d4a08e99c3213c2795f8f43eb442da33beb50c19158ec63a4ea7dae86b0a5", 1391330304),
 }
 
 
