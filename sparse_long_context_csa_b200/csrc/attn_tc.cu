@@ -70,6 +70,8 @@ struct TcParams {
   double inv_freq[64];  // theta^(-2k/R), k < R/2
   int64_t nrows;        // B * Sq queries
   int64_t nitems;       // work items = queries x key splits
+  int tma_win;          // the window rows are a plain [B, kv_rows, D] tensor: map_win covers it
+  int tma_pool;         // every visible pool entry is a key (no index lists): map_pool covers the pool
 };
 
 struct Smem {
@@ -115,7 +117,8 @@ __device__ __forceinline__ bool wait_ok(uint64_t* bar, uint32_t parity) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ TcParams P) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_win,
+                   const __grid_constant__ CUtensorMap map_pool, const __grid_constant__ TcParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const AttnArgs& a = P.a;
   const int D = a.D;
@@ -155,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tc::prefetch_tensormap(&map_q);
+    if (P.tma_win) tc::prefetch_tensormap(&map_win);
+    if (P.tma_pool) tc::prefetch_tensormap(&map_pool);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -275,6 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t kbase = tc::smem_u32(smem + L.k);
     const uint32_t qbase = tc::smem_u32(smem + L.q);
     const uint32_t pbase = tc::smem_u32(smem + L.p);
+    // Descriptors differ between MMAs only in their start address (bits 0-13, in 16-byte
+    // units), so each is formed once and stepped by adding the offset.
+    const uint64_t dK = tc::sdesc_sw128(kbase, 16, 1024);        // K tile, K-major (S^T A)
+    const uint64_t dQ = tc::sdesc_sw128(qbase, 16, 1024);        // q, K-major (S^T B)
+    const uint64_t dV = tc::sdesc_sw128(kbase, 16384, 1024);     // K tile, MN-major (PV A)
+    const uint64_t dP = tc::sdesc_sw128(pbase, 16384, 1024);     // P^T, MN-major (PV B)
     uint32_t g = 0;
     bool ok = true;
     for (int64_t n = 0; n < nq_cta && ok; ++n) {
@@ -301,12 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::fence_proxy_async_smem();  // cp.async wrote the chunk through the generic proxy
           tc::tc_fence_after();
           if (lane == 0) {
+            const uint64_t ac = dK + (uint64_t)(c * 1024), bc = dQ + (uint64_t)(c * 512);
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              const uint64_t ad = tc::sdesc_sw128(kbase + c * 16384 + kq * 32, 16, 1024);
-              const uint64_t bd = tc::sdesc_sw128(qbase + c * 8192 + kq * 32, 16, 1024);
-              tc::umma_f16(tS, ad, bd, idS, (c > 0 || kq > 0) ? 1u : 0u);
-            }
+            for (int kq = 0; kq < 4; ++kq)
+              tc::umma_f16(tS, ac + 2 * kq, bc + 2 * kq, idS, (c > 0 || kq > 0) ? 1u : 0u);
           }
           __syncwarp();
         }
@@ -326,11 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tc_fence_after();
           if (lane == 0) {
             for (int j = 0; j < nvt; ++j) {
-              for (int kk = 0; kk < nsteps; ++kk) {
-                const uint64_t ad = tc::sdesc_sw128(kbase + (2 * j) * 16384 + kk * 2048, 16384, 1024);
-                const uint64_t bd = tc::sdesc_sw128(pbase + kk * 2048, 16384, 1024);
-                tc::umma_f16(tO + 64 * j, ad, bd, idO, (i > 0 || kk > 0) ? 1u : 0u);
-              }
+              const uint64_t aj = dV + (uint64_t)(j * 2048);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                if (kk < nsteps) tc::umma_f16(tO + 64 * j, aj + 128 * kk, dP + 128 * kk, idO, (i > 0 || kk > 0) ? 1u : 0u);
             }
             tc::umma_commit(&ms->odone);
           }
@@ -374,6 +382,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k0 = (d->tile0 + i) * kTile;
       const int nvalid = min(kTile, nw4 + npool - k0);
       const int nk = (nvalid + 15) & ~15;
+      // A tile whose keys are all window rows, or all pool entries taken in order (no index
+      // list), is one run of 128 consecutive rows: TMA boxes of 64 channels x 128 rows land it
+      // in the same 128B-swizzled layout (rows past the keys are masked; rows past the
+      // tensor's end read zeros).
+      const bool all_win = k0 + kTile <= nw4 || npool == 0;
+      const bool all_pool = k0 >= nw4;
+      const CUtensorMap* tmap = nullptr;
+      int row0 = 0;
+      if (all_win && P.tma_win) {
+        tmap = &map_win;
+        row0 = b * a.kv_rows + wlo + k0;
+      } else if (all_pool && P.tma_pool) {
+        tmap = &map_pool;
+        row0 = b * a.P_cap + (k0 - nw4);
+      }
+      if (tmap) {
+        if (gcopy > 0 && !wait_ok(&ms->odone, (gcopy - 1) & 1)) ms->abort_flag = 1;
+        for (int c = 0; c < nch; ++c) {
+          if (ct == 0) {
+            tc::mbar_arrive_expect_tx(&ms->cfull[c], 16384u);
+            tc::tma_load_2d(smem + L.k + c * 16384, tmap, c * 64, row0, &ms->cfull[c]);
+          } else {
+            tc::mbar_arrive(&ms->cfull[c]);
+          }
+        }
+        return;
+      }
       const __nv_bfloat16* src[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -757,12 +792,20 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   P.nrows = rows;
   P.nitems = rows * P.a.nsplit;
   for (int k = 0; k < 64; ++k) P.inv_freq[k] = (a.R > 0 && k < a.R / 2) ? pow((double)a.theta, -2.0 * k / a.R) : 0.0;
+  // maps for tiles of consecutive rows: the window rows when they are not a ring, the pool
+  // when there are no index lists (row coordinates stay below 2^31)
+  CUtensorMap mwin = mq, mpool = mq;
+  const int64_t win_rows = (int64_t)a.B * a.kv_rows, pool_rows = (int64_t)a.B * a.P_cap;
+  P.tma_win = a.kv_win && a.n_win > 0 && !a.win_ring && win_rows + kTile < (1ll << 31) &&
+              make_row_map(&mwin, a.kv_win, a.D, win_rows, kTile);
+  P.tma_pool = a.pool && !a.idx && a.P_cap > 0 && pool_rows + kTile < (1ll << 31) &&
+               make_row_map(&mpool, a.pool, a.D, pool_rows, kTile);
   const Smem L = smem_layout(a.D);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   const int nsm = num_sms();
   const int64_t grid = P.nitems < nsm ? P.nitems : nsm;
-  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mq, P);
+  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mq, mwin, mpool, P);
   note_launch();
   if (P.a.nsplit > 1) {
     attn_split_combine_kernel<<<(unsigned)(rows * kH), 128, 0, st>>>(P.a, P);
