@@ -64,7 +64,9 @@ def part_work(w, q_index):
 
     attention: H x keys x (D + dv) x 2 FLOPs; bytes = q + out + index lists + the K=V rows
       each sequence needs once (prefill: every rotated token row and pool entry; decode:
-      the gathered rows of its one query).
+      the gathered rows of its one query); when the attention selects the index lists itself
+      (CSA prefill, dsv4_sparse_mqa_attn_scores) also the fp32 score rows it reads, and there
+      is no topk part.
     indexer_scores: visible entries x nI x cI x 2 FLOPs; bytes = the indexer pool once per
       sequence + qI + wI + the fp32 score rows written.
     indexer_topk (decode: scores and selection in one kernel): the same FLOPs; bytes = the
@@ -102,8 +104,12 @@ def part_work(w, q_index):
         kv_bytes = keys * w.D * e
     else:
         kv_bytes = w.B * (w.S + w.P_cap) * w.D * e
+    # the attention selects the lists itself (dsv4_sparse_mqa_attn_scores' fused condition, the
+    # same test as harness.selects_in_attention)
+    selects = w.kind == "csa" and w.dtype == "bf16" and 0 < w.P_cap <= 2048 and 0 < w.topk <= 512
     work = {"attention": (keys * w.H * (w.D + w.dv) * 2.0,
-                          nq * w.H * (w.D + w.dv) * e + kv_bytes + (nq * w.topk * 4 if w.topk else 0))}
+                          nq * w.H * (w.D + w.dv) * e + kv_bytes + (nq * w.topk * 4 if w.topk else 0)
+                          + (vis.sum() * 4 if selects else 0.0))}
     if w.nI > 0:
         pool_once = float(w.B) * float(vis.reshape(w.B, -1).max(axis=1).mean()) * w.cI * e
         if w.kind == "decode":
@@ -113,7 +119,8 @@ def part_work(w, q_index):
         else:
             work["indexer_scores"] = (vis.sum() * w.nI * w.cI * 2.0,
                                       pool_once + nq * w.nI * (w.cI * e + 4) + vis.sum() * 4)
-            work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
+            if not selects:
+                work["topk"] = (0.0, vis.sum() * 4 + nq * w.topk * 4)
     if w.kind != "decode":
         ch = w.D + (w.cI if w.nI else 0)
         rows_in = w.B * w.S * ch * e * (2 if w.m > 1 else 1)
@@ -168,11 +175,13 @@ NCU_TRAFFIC = {
     # window 128): dram__bytes_read.sum 564.4 MB + dram__bytes_write.sum 495.2 MB.
     ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "0ce8b3b519e30df26ca83448c5d229fa594bc968d4f9a46cb189875cf8346263", 1059631872),
     # ncu --set full, one launch of the CSA decode step (64 queries, pool 32768, top-2048): the fused
-    # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.5 MB.
-    ("csa_decode_bf16", "indexer_topk"): (_INDEXER_SOURCE, "228d6bc7b952cb7e18ac0173d08a4c71bd602164a3e3e02af47dcdba5dc1df87", 539299328),
+    # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.5 MB.  (Re-keyed
+    # when internal.h gained the attention's score-row fields; nothing this kernel compiles changed.)
+    ("csa_decode_bf16", "indexer_topk"): (_INDEXER_SOURCE, "541c61adf79361fd06ae7967948791f5445162b791cffab2b4b4ae195c364db7", 539299328),
     # ncu --set full, both launches of one output-projection step (o_a_proj, then o_b_proj; the
-    # part is the two launches): 608.2 + 117.7 + 604.0 + 61.5 MB.
-    ("out_proj_bf16", "out_proj"): (_OUT_PROJ_SOURCE, "272d4a08e99c3213c2795f8f43eb442da33beb50c19158ec63a4ea7dae86b0a5", 1391330304),
+    # part is the two launches): 608.2 + 117.7 + 604.0 + 61.5 MB.  (Re-keyed when internal.h gained
+    # the attention's score-row fields; nothing this kernel compiles changed.)
+    ("out_proj_bf16", "out_proj"): (_OUT_PROJ_SOURCE, "46c2805ba7084d9716b7a12a62394346cdbf6c5ee751bba21f79f340f4959c99", 1391330304),
 }
 
 

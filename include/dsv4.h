@@ -244,6 +244,26 @@ dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* params, const void* q, const
                                  void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * dsv4_topk_select followed by dsv4_sparse_mqa_attn, in one call ([V4] "Hybrid attention
+ * (§2.3)", CSA item: the indexer's top index_topk entries of each query go straight into core
+ * attention).  Same results as the two calls, bit for bit in idx:
+ *   idx[b,s,:] = the min(topk, vis) entries w < vis with the highest scores[b*Sq+s, w], in
+ *                ascending entry order, then -1 (ties: lower w wins; -0 equals +0),
+ *   out        = dsv4_sparse_mqa_attn(params, q, kv_win, pool, idx, sink, qpos, q_index, ...).
+ *   scores  [B*Sq, P_cap] f32   as written by dsv4_indexer_scores; entries w < vis are read
+ *   idx     [B,Sq,topk] int32   out (caller-owned): the selected lists
+ *   other arguments as for dsv4_sparse_mqa_attn (pool is required)
+ * For bf16 with P_cap <= 2048 and topk <= 512 the attention kernel selects each query's list
+ * from its score row itself (kept in shared memory; no selection launch, no list read back);
+ * otherwise the call runs the two kernels.  Validates on the host (DSV4_ERR_ARG / _SHAPE /
+ * _ALIGN) before any launch; asynchronous on `stream`.
+ */
+dsv4_status dsv4_sparse_mqa_attn_scores(const dsv4_params* params, const void* q, const void* kv_win,
+                                        const void* pool, const float* scores, const float* sink,
+                                        const int64_t* qpos, const int32_t* q_index, int32_t* idx,
+                                        void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * One CSA layer in prefill (Sq == S, query s at cache index s, RoPE position pos[b,s]):
  * compress kv -> pool (rotated) and kv_rot (window keys), compress kI -> poolI,
  * indexer + top-k -> idx, sparse attention -> out.  With m == 1, overlap == 0,

@@ -22,7 +22,7 @@ EXPORTED = ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "ds
             "dsv4_hca_layer", "dsv4_workspace_bytes", "dsv4_status_string", "dsv4_version",
             "dsv4_launch_count", "dsv4_indexer_topk_noalloc", "dsv4_device_check", "dsv4_indexer_scores",
             "dsv4_topk_select", "dsv4_decode_append", "dsv4_grouped_out_proj", "dsv4_set_index_checks",
-            "dsv4_index_checks")
+            "dsv4_index_checks", "dsv4_sparse_mqa_attn_scores")
 
 
 class Dsv4Error(RuntimeError):
@@ -63,6 +63,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_topk_select.argtypes = [P, vp, vp, vp, vp]
     lib.dsv4_decode_append.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.dsv4_sparse_mqa_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsv4_sparse_mqa_attn_scores.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsv4_csa_layer.argtypes = [P] + [vp] * 17 + [sz, vp]
     lib.dsv4_hca_layer.argtypes = [P] + [vp] * 10 + [sz, vp]
     lib.dsv4_grouped_out_proj.argtypes = [P, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -79,7 +80,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.dsv4_device_check.restype = ctypes.c_int
     for fn in ("dsv4_compress_kv", "dsv4_indexer_topk", "dsv4_sparse_mqa_attn", "dsv4_csa_layer",
                "dsv4_hca_layer", "dsv4_indexer_topk_noalloc", "dsv4_indexer_scores", "dsv4_topk_select",
-               "dsv4_decode_append", "dsv4_grouped_out_proj"):
+               "dsv4_decode_append", "dsv4_grouped_out_proj", "dsv4_sparse_mqa_attn_scores"):
         getattr(lib, fn).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -164,6 +165,15 @@ def dsv4_sparse_mqa_attn(params, q, kv_win, pool, idx, sink, qpos, q_index, out,
     _check("dsv4_sparse_mqa_attn", load().dsv4_sparse_mqa_attn(
         ctypes.byref(params), _ptr(q), _ptr(kv_win), _ptr(pool), _ptr(idx), _ptr(sink), _ptr(qpos),
         _ptr(q_index), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def dsv4_sparse_mqa_attn_scores(params, q, kv_win, pool, scores, sink, qpos, q_index, idx, out, workspace=None,
+                                ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None and workspace is not None \
+        else (ws_bytes or 0)
+    _check("dsv4_sparse_mqa_attn_scores", load().dsv4_sparse_mqa_attn_scores(
+        ctypes.byref(params), _ptr(q), _ptr(kv_win), _ptr(pool), _ptr(scores), _ptr(sink), _ptr(qpos),
+        _ptr(q_index), _ptr(idx), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def dsv4_csa_layer(params, q, kv, z, bias, qI, wI, kI, zI, biasI, sink, pos, out, pool, poolI, kv_rot, idx,

@@ -48,6 +48,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 #include "tc_ptx.cuh"
 
 namespace dsv4 {
@@ -64,6 +65,9 @@ constexpr int kMaxChunks = 9;  // D <= 576
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
 constexpr uint32_t kWaitLimit = 1u << 20;  // mbarrier polls before a wait gives up
+constexpr int kSelKeys = 2048;  // selection inside the kernel: score rows of at most this many entries
+constexpr int kSelK = 512;      // ... and index lists of at most this many slots
+constexpr uint32_t kMiscBytes = 8192;
 
 struct TcParams {
   AttnArgs a;
@@ -86,7 +90,7 @@ __host__ __device__ inline Smem smem_layout(int D) {
   const bool alias = D > 512;  // P^T reuses the last K chunk (those channels are not values)
   s.p = alias ? s.k + (nch - 1) * 16384 : s.k + nch * 16384;
   s.misc = alias ? s.k + nch * 16384 : s.p + 16384;
-  s.total = s.misc + 4096;
+  s.total = s.misc + kMiscBytes;
   return s;
 }
 
@@ -94,6 +98,7 @@ struct QDesc {
   int64_t qrow, item;
   int t, vis, wlo, nw, nw4, npool, ntiles, tile0;  // this item's tiles: [tile0, tile0 + ntiles)
   float cs[64], sn[64];  // RoPE table at the query position
+  int16_t sidx[kSelK];   // the query's index list when the kernel selects it from a score row
 };
 
 struct Misc {
@@ -108,12 +113,120 @@ struct Misc {
   float fac[kH];
   float red[4][kH];
   float inv_l[kH];
+  uint32_t sel_hist[256];  // radix histogram of the prep warp's selection
   QDesc desc[2];
 };
-static_assert(sizeof(Misc) <= 4096, "misc block exceeds its reservation");
+static_assert(sizeof(Misc) <= kMiscBytes, "misc block exceeds its reservation");
 
 __device__ __forceinline__ bool wait_ok(uint64_t* bar, uint32_t parity) {
   return tc::mbar_wait(bar, parity, kWaitLimit);
+}
+
+// One warp's top-K of the n scores sc[0..n), n <= kSelKeys, K <= kSelK: the same list as
+// dsv4_topk_select ("DeepSeek-V4" doc, Hybrid attention (§2.3), CSA item, eq. 17: the
+// index_topk highest-scoring entries; among equal scores the lower entry wins, -0 equals +0):
+// the kept entries in ascending order in sidx[0..min(K, n)), then -1 up to K.  Lane l keeps
+// the order keys of entries l + 32j in registers; the threshold key is found by 8-bit radix
+// digits of (key - smallest key), from the highest bit in which the keys differ, over a
+// 256-bin shared histogram; the ordered output is one pass of ballots in entry order.
+__device__ __forceinline__ void warp_select(const float* __restrict__ sc, int n, int K, int16_t* sidx,
+                                         uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  if (n <= K) {
+    for (int j = lane; j < K; j += 32) sidx[j] = (int16_t)(j < n ? j : -1);
+    __syncwarp();
+    return;
+  }
+  constexpr int kPer = kSelKeys / 32;
+  uint32_t key[kPer];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = lane + 32 * j;
+    key[j] = i < n ? order_key(sc[i]) : 0u;
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (lane + 32 * j < n) {
+      kmin = min(kmin, key[j]);
+      kmax = max(kmax, key[j]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  const uint32_t range = kmax - kmin;
+  int lo = range ? 32 - __clz(range) : 0;  // bits of (key - kmin) still to resolve: [0, lo)
+  uint32_t prefix = 0u, mask = 0u;
+  int need = K, cnt = -1;
+  while (lo > 0 && cnt != need) {
+    const int dlo = lo > 8 ? lo - 8 : 0;
+    const uint32_t dmask = (1u << (lo - dlo)) - 1u;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) hist[lane + 32 * b] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const uint32_t r = key[j] - kmin;
+      if (lane + 32 * j < n && (r & mask) == prefix) atomicAdd(&hist[(r >> dlo) & dmask], 1u);
+    }
+    __syncwarp();
+    // bins from the top: lane l owns bins 255 - 8l .. 248 - 8l
+    int c8[8], sum = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      c8[b] = (int)hist[255 - 8 * lane - b];
+      sum += c8[b];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - sum;
+    int bin = -1, rest = 0, bc = 0;
+    if (excl < need && need <= incl) {
+      int run = excl;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        if (bin < 0 && need <= run + c8[b]) {
+          bin = 255 - 8 * lane - b;
+          rest = need - run;
+          bc = c8[b];
+        }
+        run += c8[b];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, bin >= 0)) - 1;
+    bin = __shfl_sync(0xffffffffu, bin, src);
+    rest = __shfl_sync(0xffffffffu, rest, src);
+    bc = __shfl_sync(0xffffffffu, bc, src);
+    prefix |= (uint32_t)bin << dlo;
+    mask |= dmask << dlo;
+    need = rest;
+    cnt = bc;
+    lo = dlo;
+    __syncwarp();
+  }
+  // every entry above the prefix, and the `need` lowest-index entries equal to it
+  int pos_gt = 0, pos_eq = 0;
+  const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = lane + 32 * j;
+    const uint32_t r = (key[j] - kmin) & mask;
+    const bool gt = i < n && r > prefix, eq = i < n && r == prefix;
+    const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+    const int my_eq = pos_eq + __popc(beq & below);
+    const int slot = pos_gt + __popc(bgt & below) + min(my_eq, need);
+    if (gt || (eq && my_eq < need)) sidx[slot] = (int16_t)i;
+    pos_gt += __popc(bgt);
+    pos_eq += __popc(beq);
+  }
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -191,7 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!a.win_ring && wlo + nw > a.kv_rows) nw = a.kv_rows > wlo ? a.kv_rows - wlo : 0;
       // last valid slot of the index row (slots past it are skipped, holes are masked)
       int last = 0;
-      if (a.idx) {
+      if (a.scores) {
+        // select the index list from the score row (entries w < vis)
+        warp_select(a.scores + qrow * a.P_cap, vis, a.topk, d->sidx, ms->sel_hist);
+        last = min(a.topk, vis);
+        if (a.idx_out)
+          for (int k = lane; k < a.topk; k += 32) a.idx_out[qrow * a.topk + k] = d->sidx[k];
+      } else if (a.idx) {
         const int32_t* ir = a.idx + qrow * a.topk;
         for (int k = lane; k < a.topk; k += 32) {
           const int w = ir[k];
@@ -376,6 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const __nv_bfloat16* win_base =
           static_cast<const __nv_bfloat16*>(a.kv_win) + (int64_t)b * (a.win_ring ? a.win_ring : a.kv_rows) * D;
       const __nv_bfloat16* pool_base = static_cast<const __nv_bfloat16*>(a.pool) + (int64_t)b * a.P_cap * D;
+      // index list: selected in this kernel (shared memory) or given (global)
+      const int16_t* irs = a.scores ? d->sidx : nullptr;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
       const int cu = ct & 7;
@@ -416,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kr = k0 + r;
         if (kr >= nw4 && npool > 0) {
           const int p = kr - nw4;
-          const int w = p < npool ? (ir ? ir[p] : p) : -1;
+          const int w = p < npool ? (irs ? (int)irs[p] : ir ? ir[p] : p) : -1;
           src[j] = pool_base + (int64_t)((w >= 0 && w < vis) ? w : 0) * D + cu * 8;
         } else {
           const int jj = kr < nw ? wlo + kr : wlo;
@@ -445,6 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const QDesc* d = &ms->desc[slot];
       const int64_t qrow = d->qrow;
       const int ntiles = d->ntiles, nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis;
+      const int16_t* irs = a.scores ? d->sidx : nullptr;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       if (!first_copied && ntiles > 0) copy_tile(d, 0, g);
       first_copied = false;
@@ -462,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int p = k - nw4;
           if (p < npool) {
-            const int w = ir ? ir[p] : p;
+            const int w = irs ? (int)irs[p] : ir ? ir[p] : p;
             valid = w >= 0 && w < vis;
           } else {
             valid = false;
@@ -771,6 +893,11 @@ cudaError_t take_attn_tc_error(int* code) {
   return e;
 }
 
+bool attn_tc_selects(const AttnArgs& a, int dtype) {
+  return a.P_cap >= 1 && a.P_cap <= kSelKeys && a.topk >= 1 && a.topk <= kSelK && a.pool &&
+         attn_tc_supported(a, dtype);
+}
+
 bool attn_tc_supported(const AttnArgs& a, int dtype) {
   if (dtype != DSV4_BF16 || a.H != kH) return false;
   if (a.D % 64 != 0 || a.D < 128 || a.D > 576) return false;
@@ -798,7 +925,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   const int64_t win_rows = (int64_t)a.B * a.kv_rows, pool_rows = (int64_t)a.B * a.P_cap;
   P.tma_win = a.kv_win && a.n_win > 0 && !a.win_ring && win_rows + kTile < (1ll << 31) &&
               make_row_map(&mwin, a.kv_win, a.D, win_rows, kTile);
-  P.tma_pool = a.pool && !a.idx && a.P_cap > 0 && pool_rows + kTile < (1ll << 31) &&
+  P.tma_pool = a.pool && !a.idx && !a.scores && a.P_cap > 0 && pool_rows + kTile < (1ll << 31) &&
                make_row_map(&mpool, a.pool, a.D, pool_rows, kTile);
   const Smem L = smem_layout(a.D);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);

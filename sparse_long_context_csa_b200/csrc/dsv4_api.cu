@@ -17,6 +17,7 @@ void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_re
 namespace {
 
 constexpr size_t kScoresBudget = 256ull << 20;  // fp32 score rows kept per indexer chunk
+constexpr int64_t kSplitChunkRows = 65535;       // query rows per launch of the split indexer calls
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -133,9 +134,13 @@ dsv4_status run_indexer(const dsv4_params* p, const void* qI, const float* wI, c
   return from_cuda(launch_indexer_topk(a, p->dtype, as_stream(stream)));
 }
 
+// Attention with given index lists (idx), every visible entry (idx and scores NULL), or lists
+// the tensor-core kernel selects from score rows (scores, written to idx_out; the caller has
+// checked attn_tc_selects).
 dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
                      const int32_t* idx, const float* sink, const int64_t* qpos, const int32_t* q_index,
-                     void* out, void* workspace, size_t ws_bytes, void* stream) {
+                     void* out, void* workspace, size_t ws_bytes, void* stream, const float* scores = nullptr,
+                     int32_t* idx_out = nullptr) {
   AttnArgs a{};
   a.B = p->B; a.Sq = p->Sq; a.H = p->H; a.D = p->D; a.R = p->R; a.dv = p->dv; a.n_win = p->n_win;
   a.win_ring = p->win_ring; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk; a.rope_q = p->rope_q;
@@ -144,12 +149,15 @@ dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, co
   a.out = out;
   a.part = nullptr;
   a.nsplit = 1;
+  a.scores = scores;
+  a.idx_out = idx_out;
   const int64_t rows = (int64_t)p->B * p->Sq;
   if (rows == 0) return DSV4_OK;
   if (idx && index_checks_on()) {
     const cudaError_t e = launch_index_check(idx, q_index, rows, p->Sq, p->topk, p->m, p->P_cap, as_stream(stream));
     if (e != cudaSuccess) return from_cuda(e);
   }
+  if (scores && !attn_tc_selects(a, p->dtype)) return DSV4_ERR_SHAPE;
   if (attn_tc_supported(a, p->dtype)) {
     // few queries: split each query's keys over several CTAs when a workspace is given
     const size_t need = attn_split_bytes(rows, attn_keys_estimate(p), p->dv);
@@ -160,6 +168,14 @@ dsv4_status run_attn(const dsv4_params* p, const void* q, const void* kv_win, co
     return from_cuda(launch_attn_tc(a, as_stream(stream)));
   }
   return from_cuda(launch_attn_simt(a, p->dtype, as_stream(stream)));
+}
+
+// The tensor-core attention can select each query's index list from its score row itself.
+bool attn_selects(const dsv4_params* p, const void* pool) {
+  AttnArgs a{};
+  a.B = p->B; a.Sq = p->Sq; a.H = p->H; a.D = p->D; a.R = p->R; a.dv = p->dv; a.n_win = p->n_win;
+  a.win_ring = p->win_ring; a.m = p->m; a.P_cap = p->P_cap; a.topk = p->topk; a.pool = pool;
+  return attn_tc_selects(a, p->dtype);
 }
 
 dsv4_status check_attn_ptrs(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
@@ -285,8 +301,6 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_params* p, const void* qI, cons
 }
 
 // Rows of one launch of the split entry points (the score grids' y extents stay below 65536).
-constexpr int64_t kSplitChunkRows = 65535;
-
 dsv4_status dsv4_indexer_scores(const dsv4_params* p, const void* qI, const float* wI, const void* poolI,
                                 const int32_t* q_index, float* scores, void* stream) {
   dsv4_status st = check_common(p);
@@ -346,6 +360,25 @@ dsv4_status dsv4_sparse_mqa_attn(const dsv4_params* p, const void* q, const void
   return run_attn(p, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace, ws_bytes, stream);
 }
 
+dsv4_status dsv4_sparse_mqa_attn_scores(const dsv4_params* p, const void* q, const void* kv_win, const void* pool,
+                                        const float* scores, const float* sink, const int64_t* qpos,
+                                        const int32_t* q_index, int32_t* idx, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  dsv4_status st = check_common(p);
+  if (st != DSV4_OK) return st;
+  if ((st = check_attn(p)) != DSV4_OK) return st;
+  if (!scores || !idx) return DSV4_ERR_ARG;
+  if (p->topk < 1 || p->P_cap < 1) return DSV4_ERR_SHAPE;
+  if ((st = check_attn_ptrs(p, q, kv_win, pool, idx, sink, qpos, q_index, out)) != DSV4_OK) return st;
+  if (!aligned16(scores)) return DSV4_ERR_ALIGN;
+  if (!q_index && p->Sq > p->S) return DSV4_ERR_SHAPE;
+  if (attn_selects(p, pool))
+    return run_attn(p, q, kv_win, pool, nullptr, sink, qpos, q_index, out, workspace, ws_bytes, stream, scores, idx);
+  // otherwise the two calls this one stands for
+  if ((st = dsv4_topk_select(p, scores, q_index, idx, stream)) != DSV4_OK) return st;
+  return run_attn(p, q, kv_win, pool, idx, sink, qpos, q_index, out, workspace, ws_bytes, stream);
+}
+
 dsv4_status dsv4_csa_layer(const dsv4_params* p, const void* q, const void* kv, const void* z, const float* bias,
                            const void* qI, const float* wI, const void* kI, const void* zI, const float* biasI,
                            const float* sink, const int64_t* pos, void* out, void* pool, void* poolI,
@@ -369,6 +402,18 @@ dsv4_status dsv4_csa_layer(const dsv4_params* p, const void* q, const void* kv, 
 
   if ((st = run_compress(p, p->D, kv, z, bias, pos, 1, pool, kv_rot, stream)) != DSV4_OK) return st;
   if ((st = run_compress(p, p->cI, kI, zI, biasI, pos, 0, poolI, nullptr, stream)) != DSV4_OK) return st;
+  const int64_t rows = (int64_t)p->B * p->Sq;
+  if (attn_selects(p, pool) && scores_cap / sizeof(float) / (size_t)p->P_cap >= (size_t)rows &&
+      rows <= kSplitChunkRows) {
+    // every score row at once, then the attention selects each query's list itself
+    IndexerArgs ia{};
+    ia.B = p->B; ia.Sq = p->Sq; ia.nI = p->nI; ia.cI = p->cI; ia.m = p->m; ia.P_cap = p->P_cap; ia.topk = p->topk;
+    ia.qI = qI; ia.wI = wI; ia.poolI = poolI; ia.scores = reinterpret_cast<float*>(scores); ia.rows_per_chunk = rows;
+    const cudaError_t e = launch_indexer_scores(ia, p->dtype, 0, rows, as_stream(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+    return run_attn(p, q, kv_rot, pool, nullptr, sink, pos, nullptr, out, nullptr, 0, stream,
+                    reinterpret_cast<const float*>(scores), idx_buf);
+  }
   if ((st = run_indexer(p, qI, wI, poolI, nullptr, idx_buf, scores, scores_cap, stream)) != DSV4_OK) return st;
   return run_attn(p, q, kv_rot, pool, idx_buf, sink, pos, nullptr, out, nullptr, 0, stream);
 }

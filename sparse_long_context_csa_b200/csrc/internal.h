@@ -93,6 +93,10 @@ struct AttnArgs {
   void* out;
   float* part;  // split-over-keys partials (workspace) or nullptr
   int nsplit;   // key splits per query (1 = no split)
+  // Score rows [B*Sq, P_cap] f32 (idx then NULL): each query's index list is selected from its
+  // row inside the attention kernel, as dsv4_topk_select would, and written to idx_out.
+  const float* scores;
+  int32_t* idx_out;
 };
 // Key splits per query used by the tensor-core attention for B*Sq queries attending about
 // keys_per_query keys each (a pure function of the sizes, so that the workspace size is one
@@ -102,6 +106,8 @@ size_t attn_split_bytes(int64_t rows, int64_t keys_per_query, int dv);
 cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 // Tensor-core (tcgen05) path; returns cudaErrorNotSupported when the shape is not covered.
 bool attn_tc_supported(const AttnArgs& a, int dtype);
+// The tensor-core kernel can select the index lists from score rows (a.scores) itself.
+bool attn_tc_selects(const AttnArgs& a, int dtype);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);
 // Read and clear the tensor-core kernel's error word (non-zero: a bounded wait gave up).
 cudaError_t take_attn_tc_error(int* code);

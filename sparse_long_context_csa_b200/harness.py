@@ -182,12 +182,19 @@ def step_input_keys(w) -> list:
     return keys
 
 
+def selects_in_attention(w) -> bool:
+    """CSA prefill whose score rows are short enough for the attention kernel to select each
+    query's index list itself (dsv4_sparse_mqa_attn_scores: bf16, P_cap <= 2048, topk <= 512)."""
+    return w.kind == "csa" and w.dtype == "bf16" and 0 < w.P_cap <= 2048 and 0 < w.topk <= 512
+
+
 def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
-    """The same step as ``step`` issued entry point by entry point: for prefill the indexer as
-    its two halves (dsv4_indexer_scores into ``o["scores"]``, then dsv4_topk_select), the same
-    kernels on the same data; for decode dsv4_indexer_topk, whose one kernel scores and
-    selects.  ``events`` maps names of ``PARTS`` to (start, end) CUDA
-    event pairs recorded on ``stream`` around that part."""
+    """The same step as ``step`` issued entry point by entry point: for prefill the indexer
+    scores (dsv4_indexer_scores into ``o["scores"]``), then either the selection inside the
+    attention (dsv4_sparse_mqa_attn_scores, as dsv4_csa_layer does when the rows are short) or
+    dsv4_topk_select and dsv4_sparse_mqa_attn; for decode dsv4_indexer_topk, whose one kernel
+    scores and selects.  The same kernels on the same data as ``step``.  ``events`` maps names
+    of ``PARTS`` to (start, end) CUDA event pairs recorded on ``stream`` around that part."""
     ws = o.get("workspace")
 
     def mark(name, k):
@@ -223,13 +230,17 @@ def step_parts(w, params, x: dict, o: dict, stream=None, events=None) -> None:
         mark("indexer_scores", 0)
         abi.dsv4_indexer_scores(params, x["qI"], x["wI"], poolI, q_index, o["scores"], stream=stream)
         mark("indexer_scores", 1)
-        mark("topk", 0)
-        abi.dsv4_topk_select(params, o["scores"], q_index, o["idx"], stream=stream)
-        mark("topk", 1)
+        if not selects_in_attention(w):
+            mark("topk", 0)
+            abi.dsv4_topk_select(params, o["scores"], q_index, o["idx"], stream=stream)
+            mark("topk", 1)
     mark("attention", 0)
     if w.kind == "decode":
         abi.dsv4_sparse_mqa_attn(params, x["q"], x["win"], x["pool"], o["idx"], x["sink"], x["qpos"],
                                  x["q_index"], o["out"], ws, stream=stream)
+    elif w.nI > 0 and selects_in_attention(w):
+        abi.dsv4_sparse_mqa_attn_scores(params, x["q"], o["kv_rot"], o["pool"], o["scores"], x["sink"], x["pos"],
+                                        None, o["idx"], o["out"], ws, stream=stream)
     else:
         abi.dsv4_sparse_mqa_attn(params, x["q"], o["kv_rot"], o.get("pool"), o.get("idx"), x["sink"], x["pos"],
                                  None, o["out"], ws, stream=stream)

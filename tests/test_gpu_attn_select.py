@@ -1,0 +1,94 @@
+"""dsv4_sparse_mqa_attn_scores: the attention that selects each query's index list from its
+score row itself ("DeepSeek-V4" doc, Hybrid attention (§2.3), CSA item: the top index_topk
+entries per query go straight into core attention) against the two calls it stands for,
+dsv4_topk_select then dsv4_sparse_mqa_attn.
+
+  index lists: bit-exact (both sides rank the same fp32 values, written here on the host;
+               rows are tie-heavy: small integers, +0 and -0, +-inf, one all-equal row),
+               and pinned to the oracle's ranking on every row;
+  outputs:     bit-exact (the same kernel over the same lists).
+Rows with fewer visible entries than topk (the list is 0..vis-1, then -1) are included.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import dsv4_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_long_context_csa_b200 import abi, harness
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    abi.load()
+    return abi, harness
+
+
+def _tie_heavy_scores(rng, n_rows, P_cap):
+    sc = rng.integers(-6, 7, size=(n_rows, P_cap)).astype(np.float32)
+    zeros = rng.random((n_rows, P_cap)) < 0.05
+    sc[zeros] = np.where(rng.random(int(zeros.sum())) < 0.5, np.float32(-0.0), np.float32(0.0))
+    sc[rng.random((n_rows, P_cap)) < 0.001] = np.inf
+    sc[rng.random((n_rows, P_cap)) < 0.001] = -np.inf
+    sc[0, :] = 3.0  # all equal: the lowest entries win
+    return sc
+
+
+def _spread_scores(rng, n_rows, P_cap):
+    """Distinct-ish fp32 scores of a narrow range (the radix digits must resolve low bits)."""
+    return (1.0 + rng.random((n_rows, P_cap)) * 1e-3).astype(np.float32)
+
+
+@pytest.mark.parametrize("B,S,m,P_cap,topk,kind", [
+    (1, 8192, 4, 2048, 512, "ties"),    # the CSA prefill shape
+    (2, 2048, 1, 2048, 512, "ties"),    # every row length up to the 2048-entry limit
+    (1, 1024, 4, 256, 128, "spread"),   # rows shorter and longer than topk, narrow score range
+    (3, 600, 2, 300, 64, "ties"),       # ragged: batch of 3, tail tiles, small topk
+])
+def test_selection_in_attention_equals_two_calls(lib, B, S, m, P_cap, topk, kind):
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_prefill_bf16"].replace(B=B, S=S, Sq=S, m=m, P_cap=P_cap, topk=topk)
+    specs = synth.tensor_specs(w)
+    q = synth.reshape(w, "q", specs["q"].full())
+    kv = synth.reshape(w, "kv", specs["kv"].full())
+    rng = np.random.default_rng(20261203 + S + topk)
+    pool = (rng.standard_normal((B, P_cap, w.D)) / np.sqrt(w.D)).astype(np.float32)
+    sink = specs["sink"].full()
+    qi, qp = synth.positions(w)
+    rows = B * S
+    sc = _tie_heavy_scores(rng, rows, P_cap) if kind == "ties" else _spread_scores(rng, rows, P_cap)
+    params = harness.params_for(w)
+    dt = harness.torch_dtype(w)
+    d_q = torch.from_numpy(q).to(dt).cuda()
+    d_kv = torch.from_numpy(kv).to(dt).cuda()
+    d_pool = torch.from_numpy(pool).to(dt).cuda()
+    d_sink = torch.from_numpy(sink).cuda()
+    d_pos = torch.from_numpy(qp).cuda()
+    d_sc = torch.from_numpy(sc).cuda()
+
+    idx1 = torch.full((B, S, topk), -7, dtype=torch.int32, device="cuda")
+    out1 = torch.empty((B, S, w.H, w.dv), dtype=dt, device="cuda")
+    abi.dsv4_topk_select(params, d_sc, None, idx1)
+    abi.dsv4_sparse_mqa_attn(params, d_q, d_kv, d_pool, idx1, d_sink, d_pos, None, out1)
+    idx2 = torch.full((B, S, topk), -7, dtype=torch.int32, device="cuda")
+    out2 = torch.empty((B, S, w.H, w.dv), dtype=dt, device="cuda")
+    abi.dsv4_sparse_mqa_attn_scores(params, d_q, d_kv, d_pool, d_sc, d_sink, d_pos, None, idx2, out2)
+    abi.dsv4_device_check()
+
+    g1, g2 = idx1.cpu().numpy(), idx2.cpu().numpy()
+    assert np.array_equal(g1, g2), "index lists differ from dsv4_topk_select"
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16)), "outputs differ from the two calls"
+    # pin the lists to the oracle's ranking, row by row
+    for r in range(rows):
+        b, s = divmod(r, S)
+        vis = O.visible_entries(s, m, P_cap)
+        ranked, _ = O.topk_select_row(sc[r, :vis], topk)
+        want = np.full(topk, -1, dtype=np.int64)
+        want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
+        assert np.array_equal(g2[b, s].astype(np.int64), want), f"row {(b, s)} (vis={vis}) differs from the oracle"
