@@ -172,8 +172,9 @@ _INDEXER_SOURCE = (("indexer_tc.cu", "\n}  // namespace\n\nbool indexer_tc_suppo
 _OUT_PROJ_SOURCE = (("out_proj.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("internal.h", None))
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
-    # window 128): dram__bytes_read.sum 564.4 MB + dram__bytes_write.sum 495.2 MB.
-    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "0ce8b3b519e30df26ca83448c5d229fa594bc968d4f9a46cb189875cf8346263", 1059631872),
+    # window 128; the kernel selects each query's index list from its score row):
+    # dram__bytes_read.sum 579.6 MB + dram__bytes_write.sum 511.7 MB.
+    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "a54fe13d9175d88c22216ab380fc2c4f3bef9006147a65baa85af78a9690ecd7", 1091308544),
     # ncu --set full, one launch of the CSA decode step (64 queries, pool 32768, top-2048): the fused
     # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.5 MB.  (Re-keyed
     # when internal.h gained the attention's score-row fields; nothing this kernel compiles changed.)

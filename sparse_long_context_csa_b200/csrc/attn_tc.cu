@@ -229,6 +229,9 @@ __device__ __forceinline__ void warp_select(const float* __restrict__ sc, int n,
   __syncwarp();
 }
 
+// kSel: the index lists are selected here from score rows (a.scores); the other
+// instantiation carries none of that code.
+template <bool kSel>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_win,
                    const __grid_constant__ CUtensorMap map_pool, const __grid_constant__ TcParams P) {
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!a.win_ring && wlo + nw > a.kv_rows) nw = a.kv_rows > wlo ? a.kv_rows - wlo : 0;
       // last valid slot of the index row (slots past it are skipped, holes are masked)
       int last = 0;
-      if (a.scores) {
+      if (kSel) {
         // select the index list from the score row (entries w < vis)
         warp_select(a.scores + qrow * a.P_cap, vis, a.topk, d->sidx, ms->sel_hist);
         last = min(a.topk, vis);
@@ -496,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           static_cast<const __nv_bfloat16*>(a.kv_win) + (int64_t)b * (a.win_ring ? a.win_ring : a.kv_rows) * D;
       const __nv_bfloat16* pool_base = static_cast<const __nv_bfloat16*>(a.pool) + (int64_t)b * a.P_cap * D;
       // index list: selected in this kernel (shared memory) or given (global)
-      const int16_t* irs = a.scores ? d->sidx : nullptr;
+      const int16_t* irs = kSel ? d->sidx : nullptr;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       const int nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis, wlo = d->wlo;
       const int cu = ct & 7;
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const QDesc* d = &ms->desc[slot];
       const int64_t qrow = d->qrow;
       const int ntiles = d->ntiles, nw = d->nw, nw4 = d->nw4, npool = d->npool, vis = d->vis;
-      const int16_t* irs = a.scores ? d->sidx : nullptr;
+      const int16_t* irs = kSel ? d->sidx : nullptr;
       const int32_t* ir = a.idx ? a.idx + qrow * a.topk : nullptr;
       if (!first_copied && ntiles > 0) copy_tile(d, 0, g);
       first_copied = false;
@@ -928,11 +931,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   P.tma_pool = a.pool && !a.idx && !a.scores && a.P_cap > 0 && pool_rows + kTile < (1ll << 31) &&
                make_row_map(&mpool, a.pool, a.D, pool_rows, kTile);
   const Smem L = smem_layout(a.D);
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  auto* kern = a.scores ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   const int nsm = num_sms();
   const int64_t grid = P.nitems < nsm ? P.nitems : nsm;
-  attn_tc_kernel<<<(unsigned)grid, kThreads, L.total, st>>>(mq, mwin, mpool, P);
+  kern<<<(unsigned)grid, kThreads, L.total, st>>>(mq, mwin, mpool, P);
   note_launch();
   if (P.a.nsplit > 1) {
     attn_split_combine_kernel<<<(unsigned)(rows * kH), 128, 0, st>>>(P.a, P);
