@@ -126,6 +126,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 constexpr int kTopkBins = 4096;        // radix digits of 12 bits
 constexpr int kTopkSmemKeys = 40960;   // keys cached in shared memory (160 KB)
+constexpr int kTopkCand = 2048;        // uncached rows: keys of the threshold digit kept in shared memory
 
 __device__ __forceinline__ uint32_t row_key(const uint32_t* keys, const float* sc, bool cached, int i) {
   return cached ? keys[i] : order_key(sc[i]);
@@ -186,12 +187,18 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* 
 // while the row is loaded, then 12 and 8 more bits over the keys that still match the
 // selected prefix (skipped once the threshold digit holds exactly the keys still needed).
 // Output: the kept entries in ascending entry order, then -1.
+// A row not cached in shared memory (cache_keys == 0) whose threshold digit holds at most
+// kTopkCand keys reads its scores three times instead of five: the histogram; one pass that
+// keeps the keys of the threshold digit (with their entries) in shared memory and counts, per
+// warp segment, the keys above that digit; the ordered write.  The remaining digits are
+// resolved over the kept keys alone, which also give each segment's counts of kept keys above
+// and equal to the threshold.
 template <int NT>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs a, int64_t row0, int cache_keys) {
-  extern __shared__ uint32_t keys[];
+  extern __shared__ uint32_t keys[];  // the row's keys (cached rows) or the kept keys (uncached rows)
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int wsum[NT / 32];
-  __shared__ int s_bin, s_rest, s_cnt;
+  __shared__ int s_bin, s_rest, s_cnt, s_ncand;
   __shared__ int wcnt_gt[NT / 32], wcnt_eq[NT / 32];
   constexpr int kWarps = NT / 32;
 
@@ -234,7 +241,73 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
   uint32_t prefix = (uint32_t)s_bin << 20, mask = 0xFFF00000u;
   int need = s_rest;
-  for (int pass = 1; pass < 3 && s_cnt != need; ++pass) {
+  const int seg = (vis + kWarps - 1) / kWarps;
+  const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
+  int n_gt = 0, n_eq = 0;  // this warp segment's keys above / equal to the final prefix
+  bool counted = false;
+  if (!cached && cache_keys == 0 && s_cnt != need && s_cnt <= kTopkCand) {
+    uint64_t* cand = reinterpret_cast<uint64_t*>(keys);
+    const uint32_t b1 = (uint32_t)s_bin;
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    // keep the threshold digit's keys; count this segment's keys above it
+    for (int base = lo; base < hi; base += 32 * 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * 32 + lane;
+        v[u] = i < hi ? sc[i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * 32 + lane;
+        if (i < hi) {
+          const uint32_t k = order_key(v[u]);
+          const uint32_t dg = k >> 20;
+          n_gt += dg > b1;
+          if (dg == b1) cand[atomicAdd(&s_ncand, 1)] = ((uint64_t)k << 32) | (uint32_t)i;
+        }
+      }
+    }
+    __syncthreads();
+    const int nc = s_ncand;
+    // the remaining 12 and 8 bits over the kept keys
+    for (int pass = 1; pass < 3 && s_cnt != need; ++pass) {
+      const int shift = pass == 1 ? 8 : 0;
+      const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
+      for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < nc; i += NT) {
+        const uint32_t k = (uint32_t)(cand[i] >> 32);
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+      }
+      __syncthreads();
+      find_digit<NT>(hist, need, wsum, &s_bin, &s_rest, &s_cnt);
+      prefix |= (uint32_t)s_bin << shift;
+      mask |= dmask << shift;
+      need = s_rest;
+    }
+    // each segment's kept keys above / equal to the final prefix
+    if (tid < kWarps) {
+      wcnt_gt[tid] = 0;
+      wcnt_eq[tid] = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < nc; i += NT) {
+      const uint32_t k = (uint32_t)(cand[i] >> 32) & mask;
+      const int sw = (int)(uint32_t)cand[i] / seg;
+      if (k > prefix) atomicAdd(&wcnt_gt[sw], 1);
+      else if (k == prefix) atomicAdd(&wcnt_eq[sw], 1);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_gt += wcnt_gt[warp];
+    n_eq = wcnt_eq[warp];
+    counted = true;
+    __syncthreads();
+  }
+  for (int pass = 1; pass < 3 && s_cnt != need && !counted; ++pass) {
     const int shift = pass == 1 ? 8 : 0;
     const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
     for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
@@ -253,18 +326,17 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   // equal to it (all of them when the loop stopped early), in ascending entry order: each
   // warp owns a contiguous segment of the row; per-warp counts, a scan over warps, then
   // ordered writes.
-  const int seg = (vis + kWarps - 1) / kWarps;
-  const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
-  int n_gt = 0, n_eq = 0;
-  for (int i = lo + lane; i < hi; i += 32) {
-    const uint32_t k = row_key(keys, sc, cached, i) & mask;
-    n_gt += k > prefix;
-    n_eq += k == prefix;
-  }
+  if (!counted) {
+    for (int i = lo + lane; i < hi; i += 32) {
+      const uint32_t k = row_key(keys, sc, cached, i) & mask;
+      n_gt += k > prefix;
+      n_eq += k == prefix;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
-    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
   }
   if (lane == 0) {
     wcnt_gt[warp] = n_gt;
@@ -381,9 +453,10 @@ cudaError_t launch_topk(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream
   // 2.83 ms; 64 decode rows: 29 -> 91 us, hence the row count).
   const int64_t rows = r1 - r0;
   const bool wide = a.P_cap > 4096 && rows < 4 * 148;
-  const size_t smem = a.P_cap > 4096 && !wide ? 0
-                      : (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
-  const int cache_keys = (int)(smem / sizeof(uint32_t));
+  const bool uncached = a.P_cap > 4096 && !wide;
+  const size_t smem = uncached ? (size_t)kTopkCand * sizeof(uint64_t)
+                               : (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
+  const int cache_keys = uncached ? 0 : (int)(smem / sizeof(uint32_t));
   cudaError_t e = wide ? cudaFuncSetAttribute(topk_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
                        : cudaFuncSetAttribute(topk_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

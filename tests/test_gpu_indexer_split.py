@@ -106,6 +106,36 @@ def test_topk_select_bit_exact(lib, P_cap, topk):
         assert np.array_equal(g[s].astype(np.int64), want), f"row {s} (vis={vis}) differs from the oracle"
 
 
+@pytest.mark.parametrize("topk", [512, 2048])
+def test_topk_select_many_long_rows_bit_exact(lib, topk):
+    """Hundreds of rows longer than 4096 entries take the path that re-reads each row from its
+    scores (256 threads per row, several rows per SM): there the keys of the threshold digit
+    are kept in shared memory when there are at most 2048 of them, and the row is read three
+    times.  Rows of narrow-range distinct scores take that path; tie-heavy rows (thousands of
+    keys in one digit) the general one.  Every row against the oracle's ranking."""
+    abi, harness = lib
+    P_cap, Sq = 9000, 700
+    rng = np.random.default_rng(20261203 + topk)
+    q_index = rng.integers(0, P_cap, size=(1, Sq)).astype(np.int32)
+    q_index[0, :4] = [P_cap - 1, topk - 1, topk, 4096]
+    sc = _tie_heavy_scores(rng, Sq, P_cap)
+    spread = rng.random(Sq) < 0.5
+    spread[:2] = [False, True]
+    sc[spread] = (1.0 + rng.random((int(spread.sum()), P_cap)) * 1e-3).astype(np.float32)
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=1, Sq=Sq, S=P_cap, m=1, P_cap=P_cap, topk=topk)
+    params = harness.params_for(w)
+    idx = torch.full((1, Sq, topk), -7, dtype=torch.int32, device="cuda")
+    abi.dsv4_topk_select(params, torch.from_numpy(sc).cuda(), torch.from_numpy(q_index).cuda(), idx)
+    abi.dsv4_device_check()
+    g = idx.cpu().numpy()[0]
+    for s in range(Sq):
+        vis = O.visible_entries(int(q_index[0, s]), 1, P_cap)
+        ranked, _ = O.topk_select_row(sc[s, :vis], topk)
+        want = np.full(topk, -1, dtype=np.int64)
+        want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
+        assert np.array_equal(g[s].astype(np.int64), want), f"row {s} (vis={vis}) differs from the oracle"
+
+
 @pytest.mark.parametrize("name", ["tiny_csa_f32", "csa_decode_bf16"])
 def test_split_calls_equal_fused_call(lib, name):
     abi, harness = lib
