@@ -72,6 +72,31 @@ def test_attention_rejects_bad_arguments(abi):
     assert _attn(abi, _params(abi, m=0)) == 2
 
 
+def _attn_scores(abi, p, **over):
+    a = dict(q=FAKE, kv_win=FAKE, pool=FAKE, scores=FAKE, sink=FAKE, qpos=FAKE, q_index=None, idx=FAKE, out=FAKE)
+    a.update(over)
+    lib = abi.load()
+    return lib.dsv4_sparse_mqa_attn_scores(ctypes.byref(p) if p is not None else None, a["q"], a["kv_win"],
+                                           a["pool"], a["scores"], a["sink"], a["qpos"], a["q_index"], a["idx"],
+                                           a["out"], None, 0, None)
+
+
+def test_attention_with_selection_rejects_bad_arguments(abi):
+    """dsv4_sparse_mqa_attn_scores validates like dsv4_topk_select + dsv4_sparse_mqa_attn,
+    on the host, before any launch (every call here fails validation)."""
+    assert _attn_scores(abi, None) == 1
+    assert _attn_scores(abi, _params(abi, dtype=7)) == 4
+    assert _attn_scores(abi, _params(abi), scores=None) == 1     # the score rows are required
+    assert _attn_scores(abi, _params(abi), idx=None) == 1        # ... and the lists' buffer
+    assert _attn_scores(abi, _params(abi), pool=None) == 1       # lists need a pool
+    assert _attn_scores(abi, _params(abi), scores=FAKE + 4) == 3
+    assert _attn_scores(abi, _params(abi), idx=FAKE + 8) == 3
+    assert _attn_scores(abi, _params(abi, topk=0)) == 2
+    assert _attn_scores(abi, _params(abi, dv=256)) == 2          # rotate_out needs dv == D
+    assert _attn_scores(abi, _params(abi), q=None) == 1
+    assert _attn_scores(abi, _params(abi), qpos=None) == 1
+
+
 def test_indexer_rejects_bad_arguments(abi):
     lib = abi.load()
 

@@ -92,3 +92,40 @@ def test_selection_in_attention_equals_two_calls(lib, B, S, m, P_cap, topk, kind
         want = np.full(topk, -1, dtype=np.int64)
         want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
         assert np.array_equal(g2[b, s].astype(np.int64), want), f"row {(b, s)} (vis={vis}) differs from the oracle"
+
+
+@pytest.mark.parametrize("B,S,P_cap,topk", [(16, 8192, 2048, 512), (7, 4000, 1000, 256)])
+def test_selection_in_attention_decode_shapes(lib, B, S, P_cap, topk):
+    """One query per sequence at a spread of cache positions, the window in a ring, and a
+    workspace, so each query's keys are split over several CTAs (each split selects the same
+    list): lists and outputs bit-exact against dsv4_topk_select + dsv4_sparse_mqa_attn, lists
+    against the oracle's ranking."""
+    abi, harness = lib
+    w = synth.WORKLOADS["csa_decode_bf16"].replace(B=B, S=S, P_cap=P_cap, topk=topk, qindex_spread=min(1024, S // 4))
+    host = synth.make_inputs(w)
+    params = harness.params_for(w)
+    x = harness.to_device(w, host)
+    rng = np.random.default_rng(20261204 + B)
+    sc = _spread_scores(rng, B, P_cap)
+    sc[0] = _tie_heavy_scores(rng, 1, P_cap)[0]
+    d_sc = torch.from_numpy(sc).cuda()
+    ws = torch.empty(max(abi.dsv4_workspace_bytes(params), 256), dtype=torch.uint8, device="cuda")
+    dt = harness.torch_dtype(w)
+    idx1 = torch.full((B, 1, topk), -7, dtype=torch.int32, device="cuda")
+    out1 = torch.empty((B, 1, w.H, w.dv), dtype=dt, device="cuda")
+    abi.dsv4_topk_select(params, d_sc, x["q_index"], idx1)
+    abi.dsv4_sparse_mqa_attn(params, x["q"], x["win"], x["pool"], idx1, x["sink"], x["qpos"], x["q_index"], out1, ws)
+    idx2 = torch.full((B, 1, topk), -7, dtype=torch.int32, device="cuda")
+    out2 = torch.empty((B, 1, w.H, w.dv), dtype=dt, device="cuda")
+    abi.dsv4_sparse_mqa_attn_scores(params, x["q"], x["win"], x["pool"], d_sc, x["sink"], x["qpos"], x["q_index"],
+                                    idx2, out2, ws)
+    abi.dsv4_device_check()
+    g1, g2 = idx1.cpu().numpy(), idx2.cpu().numpy()
+    assert np.array_equal(g1, g2), "index lists differ from dsv4_topk_select"
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16)), "outputs differ from the two calls"
+    for b in range(B):
+        vis = O.visible_entries(int(host["q_index"][b, 0]), w.m, P_cap)
+        ranked, _ = O.topk_select_row(sc[b, :vis], topk)
+        want = np.full(topk, -1, dtype=np.int64)
+        want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
+        assert np.array_equal(g2[b, 0].astype(np.int64), want), f"sequence {b} (vis={vis}) differs from the oracle"
