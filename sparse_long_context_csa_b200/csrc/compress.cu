@@ -63,14 +63,16 @@ __device__ __forceinline__ float2 pool_pair(const T* __restrict__ x, const T* __
 }
 
 // RoPE of channel pair (d, d+1) when it lies in the trailing R channels; inv_freq[k] =
-// theta^(-2k/R) comes from the host, the angle pos * inv_freq[k] is formed and reduced in
-// double precision (positions up to 2^20 keep full float accuracy in cos/sin).
+// theta^(-2k/R) comes from the host, the angle pos * inv_freq[k] is formed and reduced to
+// [-pi, pi] in double precision (positions up to 2^20 keep full float accuracy), then its
+// cos/sin are taken in float.
 __device__ __forceinline__ float2 rope_pair(float2 v, int64_t pos, int d, int c, int R, const double* inv_freq) {
   const int rope_lo = c - R;
   if (d < rope_lo) return v;
-  double sd, cd;
-  sincos((double)pos * inv_freq[(d - rope_lo) / 2], &sd, &cd);
-  const float cs = (float)cd, sn = (float)sd;
+  double ang = (double)pos * inv_freq[(d - rope_lo) / 2];
+  ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;
+  float sn, cs;
+  sincosf((float)ang, &sn, &cs);
   return make_float2(v.x * cs - v.y * sn, v.x * sn + v.y * cs);
 }
 
@@ -105,14 +107,28 @@ __global__ void __launch_bounds__(256, 5) compress_kernel(const __grid_constant_
   }
 
   if (a.x_rot) {
+    // the block's rows as one list of pairs: first every row's pairs before the trailing R
+    // channels (copied), then every row's R/2 rotated pairs, so that with many rows the
+    // rotations are spread over all threads (a thread keeps no fixed pair)
     T* __restrict__ xr = static_cast<T*>(a.x_rot) + (int64_t)b * S * c;
-    const int t_hi = min((w + 1) * m, S);
-    const int npairs = c / 2;
-    for (int it = threadIdx.x; it < (t_hi - w * m) * npairs; it += blockDim.x) {
-      const int j = w * m + it / npairs;
-      const int d = 2 * (it % npairs);
-      const float2 v = rope_pair(load2<T>(x + (int64_t)j * c + d), pos[j], d, c, a.R, a.inv_freq);
-      store2<T>(xr + (int64_t)j * c + d, v.x, v.y);
+    const int t0 = w * m;
+    const int ntok = min((w + 1) * m, S) - t0;
+    const int nrp = a.R / 2;
+    const int np0 = c / 2 - nrp;
+    const int ncopy = ntok * np0;
+    for (int it = threadIdx.x; it < ntok * (np0 + nrp); it += blockDim.x) {
+      if (it < ncopy) {
+        const int64_t j = t0 + it / np0;
+        const int d = 2 * (it % np0);
+        const float2 v = load2<T>(x + j * c + d);
+        store2<T>(xr + j * c + d, v.x, v.y);
+      } else {
+        const int k = it - ncopy;
+        const int64_t j = t0 + k / nrp;
+        const int d = 2 * (np0 + k % nrp);
+        const float2 v = rope_pair(load2<T>(x + j * c + d), pos[j], d, c, a.R, a.inv_freq);
+        store2<T>(xr + j * c + d, v.x, v.y);
+      }
     }
   }
 }
