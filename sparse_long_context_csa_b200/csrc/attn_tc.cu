@@ -838,50 +838,73 @@ int num_sms() {
 
 // Merge the key splits of one (query, head): o = sum_s 2^{m_s - M} O_s / (2^{sink - M} +
 // sum_s 2^{m_s - M} l_s), then the -qpos rotation of the rope slice.  One CTA of dv/4
-// threads per (query, head); thread = 4 consecutive channels.
+// threads per (query, kCombineHeads heads); thread = 4 consecutive channels of each head, so
+// that a thread has the loads of several heads in flight (4 heads per CTA instead of 1: decode
+// attention with the combine 88.7 -> 85.2 us).
+constexpr int kCombineHeads = 4;
+
 __global__ void __launch_bounds__(128) attn_split_combine_kernel(const AttnArgs a, const TcParams P) {
-  const int64_t qrow = blockIdx.x / kH;
-  const int h = blockIdx.x % kH;
+  const int64_t qrow = blockIdx.x / (kH / kCombineHeads);
+  const int hb = (int)(blockIdx.x % (kH / kCombineHeads)) * kCombineHeads;
   const int t4 = threadIdx.x;  // channels 4*t4 .. 4*t4+3
   if (4 * t4 >= a.dv) return;
   const int64_t stride = (int64_t)kH * (a.dv + 2);
   const float* base = a.part + qrow * a.nsplit * stride;
-  const float sink2 = a.sink[h] * kLog2e;
-  float M = sink2;
-  for (int sp = 0; sp < a.nsplit; ++sp) M = fmaxf(M, base[sp * stride + (int64_t)kH * a.dv + 2 * h]);
-  float L = tc::ex2(sink2 - M);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sp = 0; sp < a.nsplit; ++sp) {
-    const float* ml = base + sp * stride + (int64_t)kH * a.dv + 2 * h;
-    const float w = tc::ex2(ml[0] - M);
-    L += w * ml[1];
-    const float4 v = *reinterpret_cast<const float4*>(base + sp * stride + (int64_t)h * a.dv + 4 * t4);
-    acc.x += w * v.x;
-    acc.y += w * v.y;
-    acc.z += w * v.z;
-    acc.w += w * v.w;
-  }
-  const float inv = 1.f / L;
-  float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
   const int rope_lo = a.D - a.R;
-  if (a.rotate_out && 4 * t4 >= rope_lo) {
+  const bool rot = a.rotate_out && 4 * t4 >= rope_lo;
+  float cs[2] = {1.f, 1.f}, sn[2] = {0.f, 0.f};
+  if (rot) {
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      const int kp = (4 * t4 + e - rope_lo) >> 1;
+    for (int e = 0; e < 2; ++e) {
+      const int kp = (4 * t4 + 2 * e - rope_lo) >> 1;
       double ang = (double)a.qpos[qrow] * P.inv_freq[kp];
       ang -= rint(ang * 0.15915494309189535) * 6.283185307179586;
-      float c, sn;
-      sincosf((float)ang, &sn, &c);
-      const float x0 = x[e], x1 = x[e + 1];
-      x[e] = x0 * c + x1 * sn;
-      x[e + 1] = x1 * c - x0 * sn;
+      sincosf((float)ang, &sn[e], &cs[e]);
     }
   }
-  __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&b0);
-  pk.y = *reinterpret_cast<uint32_t*>(&b1);
-  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (qrow * kH + h) * a.dv + 4 * t4) = pk;
+  float M[kCombineHeads], L[kCombineHeads];
+  float4 acc[kCombineHeads];
+#pragma unroll
+  for (int k = 0; k < kCombineHeads; ++k) {
+    M[k] = a.sink[hb + k] * kLog2e;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int sp = 0; sp < a.nsplit; ++sp)
+#pragma unroll
+    for (int k = 0; k < kCombineHeads; ++k) M[k] = fmaxf(M[k], base[sp * stride + (int64_t)kH * a.dv + 2 * (hb + k)]);
+#pragma unroll
+  for (int k = 0; k < kCombineHeads; ++k) L[k] = tc::ex2(a.sink[hb + k] * kLog2e - M[k]);
+  for (int sp = 0; sp < a.nsplit; ++sp) {
+#pragma unroll
+    for (int k = 0; k < kCombineHeads; ++k) {
+      const float* ml = base + sp * stride + (int64_t)kH * a.dv + 2 * (hb + k);
+      const float w = tc::ex2(ml[0] - M[k]);
+      L[k] += w * ml[1];
+      const float4 v = *reinterpret_cast<const float4*>(base + sp * stride + (int64_t)(hb + k) * a.dv + 4 * t4);
+      acc[k].x += w * v.x;
+      acc[k].y += w * v.y;
+      acc[k].z += w * v.z;
+      acc[k].w += w * v.w;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kCombineHeads; ++k) {
+    const float inv = 1.f / L[k];
+    float x[4] = {acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv};
+    if (rot) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float x0 = x[2 * e], x1 = x[2 * e + 1];
+        x[2 * e] = x0 * cs[e] + x1 * sn[e];
+        x[2 * e + 1] = x1 * cs[e] - x0 * sn[e];
+      }
+    }
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&b0);
+    pk.y = *reinterpret_cast<uint32_t*>(&b1);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + (qrow * kH + hb + k) * a.dv + 4 * t4) = pk;
+  }
 }
 
 cudaError_t take_attn_tc_error(int* code) {
@@ -939,7 +962,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   kern<<<(unsigned)grid, kThreads, L.total, st>>>(mq, mwin, mpool, P);
   note_launch();
   if (P.a.nsplit > 1) {
-    attn_split_combine_kernel<<<(unsigned)(rows * kH), 128, 0, st>>>(P.a, P);
+    attn_split_combine_kernel<<<(unsigned)(rows * (kH / kCombineHeads)), 128, 0, st>>>(P.a, P);
     note_launch();
   }
   return cudaGetLastError();
