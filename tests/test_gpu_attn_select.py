@@ -129,3 +129,36 @@ def test_selection_in_attention_decode_shapes(lib, B, S, P_cap, topk):
         want = np.full(topk, -1, dtype=np.int64)
         want[:len(ranked)] = np.sort(np.asarray(ranked, dtype=np.int64))
         assert np.array_equal(g2[b, 0].astype(np.int64), want), f"sequence {b} (vis={vis}) differs from the oracle"
+
+
+@pytest.mark.parametrize("name,P_cap,topk", [("tiny_csa_f32", 128, 32), ("csa_prefill_bf16", 4096, 512)])
+def test_selection_fallback_equals_two_calls(lib, name, P_cap, topk):
+    """Where the attention kernel does not select itself (fp32, or rows longer than 2048
+    entries), dsv4_sparse_mqa_attn_scores runs dsv4_topk_select and dsv4_sparse_mqa_attn: the
+    same lists and outputs, bit for bit."""
+    abi, harness = lib
+    w0 = synth.WORKLOADS[name]
+    S = 512 if name.startswith("tiny") else 2048
+    w = w0.replace(S=S, Sq=S, m=max(1, S // P_cap), P_cap=P_cap, topk=topk)
+    specs = synth.tensor_specs(w)
+    q = synth.reshape(w, "q", specs["q"].full())
+    kv = synth.reshape(w, "kv", specs["kv"].full())
+    rng = np.random.default_rng(20261205 + P_cap)
+    pool = (rng.standard_normal((w.B, P_cap, w.D)) / np.sqrt(w.D)).astype(np.float32)
+    sink = specs["sink"].full()
+    _, qp = synth.positions(w)
+    sc = _spread_scores(rng, w.B * S, P_cap)
+    params = harness.params_for(w)
+    dt = harness.torch_dtype(w)
+    d = [torch.from_numpy(v).to(dt).cuda() for v in (q, kv, pool)]
+    d_sink, d_pos, d_sc = torch.from_numpy(sink).cuda(), torch.from_numpy(qp).cuda(), torch.from_numpy(sc).cuda()
+    idx1 = torch.full((w.B, S, topk), -7, dtype=torch.int32, device="cuda")
+    idx2 = torch.full((w.B, S, topk), -7, dtype=torch.int32, device="cuda")
+    out1 = torch.empty((w.B, S, w.H, w.dv), dtype=dt, device="cuda")
+    out2 = torch.empty((w.B, S, w.H, w.dv), dtype=dt, device="cuda")
+    abi.dsv4_topk_select(params, d_sc, None, idx1)
+    abi.dsv4_sparse_mqa_attn(params, d[0], d[1], d[2], idx1, d_sink, d_pos, None, out1)
+    abi.dsv4_sparse_mqa_attn_scores(params, d[0], d[1], d[2], d_sc, d_sink, d_pos, None, idx2, out2)
+    abi.dsv4_device_check()
+    assert torch.equal(idx1, idx2), "index lists differ"
+    assert torch.equal(out1, out2), "outputs differ"
