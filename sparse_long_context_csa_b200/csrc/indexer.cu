@@ -126,10 +126,25 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 constexpr int kTopkBins = 4096;        // radix digits of 12 bits
 constexpr int kTopkSmemKeys = 40960;   // keys cached in shared memory (160 KB)
-constexpr int kTopkCand = 2048;        // uncached rows: keys of the threshold digit kept in shared memory
 
-__device__ __forceinline__ uint32_t row_key(const uint32_t* keys, const float* sc, bool cached, int i) {
-  return cached ? keys[i] : order_key(sc[i]);
+constexpr int kTopkListBytes = 20480;  // uncached rows: the warps' lists of entries at or above the threshold digit
+constexpr uint32_t kListDigit = 0x80000000u;  // list entry flag: the entry's key is in the threshold digit
+
+// The keys of entries base + u * stride (u < 8), 0 at or past `end`: all eight loads are
+// issued before any is used, so a pass over a long row costs a few memory round trips per
+// eight keys of each thread instead of one per key.
+__device__ __forceinline__ void row_keys8(uint32_t (&k)[8], const uint32_t* keys, const float* sc, bool cached,
+                                          int base, int stride, int end) {
+  if (cached) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k[u] = base + u * stride < end ? keys[base + u * stride] : 0u;
+  } else {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = base + u * stride < end ? sc[base + u * stride] : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k[u] = order_key(v[u]);
+  }
 }
 
 // Finds the digit holding the need-th largest key of a histogram (digits scanned from the
@@ -187,20 +202,25 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* 
 // while the row is loaded, then 12 and 8 more bits over the keys that still match the
 // selected prefix (skipped once the threshold digit holds exactly the keys still needed).
 // Output: the kept entries in ascending entry order, then -1.
-// A row not cached in shared memory (cache_keys == 0) whose threshold digit holds at most
-// kTopkCand keys reads its scores three times instead of five: the histogram; one pass that
-// keeps the keys of the threshold digit (with their entries) in shared memory and counts, per
-// warp segment, the keys above that digit; the ordered write.  The remaining digits are
-// resolved over the kept keys alone, which also give each segment's counts of kept keys above
-// and equal to the threshold.
+// A row not cached in shared memory (cache_keys == 0) reads its scores twice: the histogram,
+// then one pass in which each warp lists, in entry order, the entries of its segment of the
+// row whose key is at or above the threshold digit (a flag marks those in that digit).  The
+// remaining digits, the counts and the ordered write then go over the lists alone (the keys
+// of the listed threshold-digit entries are read again).  A list that would outgrow its share
+// of shared memory sends the row to the passes over the whole row; when the threshold digit
+// holds one value only (a long run of equal scores, such as the exact zeros that ReLU leaves
+// in a one-head indexer), that value is the whole prefix and the counts come from the same
+// pass.
 template <int NT>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs a, int64_t row0, int cache_keys) {
-  extern __shared__ uint32_t keys[];  // the row's keys (cached rows) or the kept keys (uncached rows)
+  extern __shared__ __align__(16) uint32_t keys[];  // the row's keys (cached rows) or the warps' lists
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int wsum[NT / 32];
-  __shared__ int s_bin, s_rest, s_cnt, s_ncand;
+  __shared__ int s_bin, s_rest, s_cnt, s_over;
+  __shared__ uint32_t s_kmin, s_kmax;
   __shared__ int wcnt_gt[NT / 32], wcnt_eq[NT / 32];
   constexpr int kWarps = NT / 32;
+  constexpr int kCap = kTopkListBytes / 4 / kWarps;  // entries of one warp's list
 
   const int64_t row = row0 + blockIdx.x;
   const int s = (int)(row % a.Sq);
@@ -209,6 +229,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   const int K = a.topk;
   int32_t* out = a.idx + row * (int64_t)K;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned below = (1u << lane) - 1u;
 
   if (vis <= K) {
     for (int i = tid; i < K; i += NT) out[i] = i < vis ? i : -1;
@@ -218,22 +239,15 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   const bool cached = vis <= cache_keys;  // keys kept in shared memory
   for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
   __syncthreads();
-  // Eight score loads per thread are issued before any is used, so a long row costs a few
-  // memory round trips instead of one per key.
   for (int base = tid; base < vis; base += NT * 8) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = base + u * NT;
-      v[u] = j < vis ? sc[j] : 0.f;
-    }
+    uint32_t kk[8];
+    row_keys8(kk, keys, sc, false, base, NT, vis);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int j = base + u * NT;
       if (j < vis) {
-        const uint32_t k = order_key(v[u]);
-        if (cached) keys[j] = k;
-        atomicAdd(&hist[k >> 20], 1u);
+        if (cached) keys[j] = kk[u];
+        atomicAdd(&hist[kk[u] >> 20], 1u);
       }
     }
   }
@@ -244,42 +258,76 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   const int seg = (vis + kWarps - 1) / kWarps;
   const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
   int n_gt = 0, n_eq = 0;  // this warp segment's keys above / equal to the final prefix
-  bool counted = false;
-  if (!cached && cache_keys == 0 && s_cnt != need && s_cnt <= kTopkCand) {
-    uint64_t* cand = reinterpret_cast<uint64_t*>(keys);
+  bool counted = false, listed = false;
+  int len = 0;  // entries at or above the threshold digit in this warp's segment
+  uint32_t* list = keys + warp * kCap;
+  if (!cached && cache_keys == 0) {
     const uint32_t b1 = (uint32_t)s_bin;
-    if (tid == 0) s_ncand = 0;
+    // a list can outgrow its share only when the entries to list outnumber one share
+    const bool track = K - need + s_cnt > kCap;
+    if (tid == 0) {
+      s_over = 0;
+      s_kmin = 0xFFFFFFFFu;
+      s_kmax = 0u;
+    }
     __syncthreads();
-    // keep the threshold digit's keys; count this segment's keys above it
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int base = lo; base < hi; base += 32 * 8) {
-      float v[8];
+      uint32_t kk[8];
+      row_keys8(kk, keys, sc, false, base + lane, 32, hi);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = base + u * 32 + lane;
-        v[u] = i < hi ? sc[i] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = base + u * 32 + lane;
-        if (i < hi) {
-          const uint32_t k = order_key(v[u]);
-          const uint32_t dg = k >> 20;
-          n_gt += dg > b1;
-          if (dg == b1) cand[atomicAdd(&s_ncand, 1)] = ((uint64_t)k << 32) | (uint32_t)i;
+        const uint32_t dg = kk[u] >> 20;
+        const bool sel = i < hi && dg >= b1;
+        const unsigned bs = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+          const int pos = len + __popc(bs & below);
+          if (pos < kCap) list[pos] = (uint32_t)i | (dg == b1 ? kListDigit : 0u);
+          if (track && dg == b1) {
+            n_eq += 1;
+            kmin = min(kmin, kk[u]);
+            kmax = max(kmax, kk[u]);
+          }
         }
+        len += __popc(bs);
+      }
+    }
+    if (lane == 0 && len > kCap) s_over = 1;
+    if (track) {
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+      if (lane == 0 && kmin <= kmax) {
+        atomicMin(&s_kmin, kmin);
+        atomicMax(&s_kmax, kmax);
       }
     }
     __syncthreads();
-    const int nc = s_ncand;
-    // the remaining 12 and 8 bits over the kept keys
+    listed = s_over == 0;
+    if (!listed && s_cnt != need && s_kmin == s_kmax) {
+      // the threshold digit holds one value: it is the whole prefix, and the counts are done
+      prefix = s_kmin;
+      mask = 0xFFFFFFFFu;
+      n_gt = len - n_eq;
+      counted = true;
+    } else {
+      n_eq = 0;
+    }
+  }
+  if (listed) {
+    // the remaining 12 and 8 bits over the listed threshold-digit entries
     for (int pass = 1; pass < 3 && s_cnt != need; ++pass) {
       const int shift = pass == 1 ? 8 : 0;
       const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
       for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
       __syncthreads();
-      for (int i = tid; i < nc; i += NT) {
-        const uint32_t k = (uint32_t)(cand[i] >> 32);
-        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+      for (int p = lane; p < len; p += 32) {
+        const uint32_t e = list[p];
+        if (e & kListDigit) {
+          const uint32_t k = order_key(sc[e & ~kListDigit]);
+          if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+        }
       }
       __syncthreads();
       find_digit<NT>(hist, need, wsum, &s_bin, &s_rest, &s_cnt);
@@ -287,34 +335,36 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
       mask |= dmask << shift;
       need = s_rest;
     }
-    // each segment's kept keys above / equal to the final prefix
-    if (tid < kWarps) {
-      wcnt_gt[tid] = 0;
-      wcnt_eq[tid] = 0;
+    // this segment's listed keys above / equal to the final prefix (entries outside the
+    // threshold digit are above it)
+    for (int p = lane; p < len; p += 32) {
+      const uint32_t e = list[p];
+      if (e & kListDigit) {
+        const uint32_t k = order_key(sc[e & ~kListDigit]) & mask;
+        n_gt += k > prefix;
+        n_eq += k == prefix;
+      } else {
+        n_gt += 1;
+      }
     }
-    __syncthreads();
-    for (int i = tid; i < nc; i += NT) {
-      const uint32_t k = (uint32_t)(cand[i] >> 32) & mask;
-      const int sw = (int)(uint32_t)cand[i] / seg;
-      if (k > prefix) atomicAdd(&wcnt_gt[sw], 1);
-      else if (k == prefix) atomicAdd(&wcnt_eq[sw], 1);
-    }
-    __syncthreads();
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
-    n_gt += wcnt_gt[warp];
-    n_eq = wcnt_eq[warp];
+    for (int o = 16; o > 0; o >>= 1) {
+      n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+      n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
     counted = true;
-    __syncthreads();
   }
   for (int pass = 1; pass < 3 && s_cnt != need && !counted; ++pass) {
     const int shift = pass == 1 ? 8 : 0;
     const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
     for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < vis; i += NT) {
-      const uint32_t k = row_key(keys, sc, cached, i);
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+    for (int base = tid; base < vis; base += NT * 8) {
+      uint32_t kk[8];
+      row_keys8(kk, keys, sc, cached, base, NT, vis);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (base + u * NT < vis && (kk[u] & mask) == prefix) atomicAdd(&hist[(kk[u] >> shift) & dmask], 1u);
     }
     __syncthreads();
     find_digit<NT>(hist, need, wsum, &s_bin, &s_rest, &s_cnt);
@@ -327,10 +377,16 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   // warp owns a contiguous segment of the row; per-warp counts, a scan over warps, then
   // ordered writes.
   if (!counted) {
-    for (int i = lo + lane; i < hi; i += 32) {
-      const uint32_t k = row_key(keys, sc, cached, i) & mask;
-      n_gt += k > prefix;
-      n_eq += k == prefix;
+    for (int base = lo + lane; base < hi; base += 32 * 8) {
+      uint32_t kk[8];
+      row_keys8(kk, keys, sc, cached, base, 32, hi);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t k = kk[u] & mask;
+        const bool in = base + u * 32 < hi;
+        n_gt += in && k > prefix;
+        n_eq += in && k == prefix;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -351,19 +407,42 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   // output slot of an entry = (kept entries before it): kept-greater before it plus the kept
   // ties before it (ties are kept while their rank among ties is below `need`)
   int pos_gt = gt_before, pos_eq = eq_before;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t k = i < hi ? row_key(keys, sc, cached, i) & mask : 0u;
-    const bool gt = i < hi && k > prefix;
-    const bool eq = i < hi && k == prefix;
-    const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
-    const unsigned below = (1u << lane) - 1u;
-    const int my_eq_rank = pos_eq + __popc(beq & below);
-    const int kept_eq_before = min(my_eq_rank, need);
-    const int slot = pos_gt + __popc(bgt & below) + kept_eq_before;
-    if ((gt || (eq && my_eq_rank < need)) && slot < K) out[slot] = i;
-    pos_gt += __popc(bgt);
-    pos_eq += __popc(beq);
+  const int gt_end = gt_before + wcnt_gt[warp];
+  if (listed) {
+    for (int base = 0; base < len; base += 32) {
+      const int p = base + lane;
+      const uint32_t e = p < len ? list[p] : 0u;
+      const bool dig = (e & kListDigit) != 0u;
+      const uint32_t k = dig ? order_key(sc[e & ~kListDigit]) & mask : 0u;
+      const bool gt = p < len && (!dig || k > prefix);
+      const bool eq = p < len && dig && k == prefix;
+      const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+      const int my_eq_rank = pos_eq + __popc(beq & below);
+      const int slot = pos_gt + __popc(bgt & below) + min(my_eq_rank, need);
+      if ((gt || (eq && my_eq_rank < need)) && slot < K) out[slot] = (int)(e & ~kListDigit);
+      pos_gt += __popc(bgt);
+      pos_eq += __popc(beq);
+    }
+    return;
+  }
+  // A warp stops once its segment's greater keys are all written and the kept ties are all
+  // behind it (a long run of one value keeps only its first `need` entries).
+  for (int base = lo; base < hi && (pos_gt < gt_end || pos_eq < need); base += 32 * 8) {
+    uint32_t kk[8];
+    row_keys8(kk, keys, sc, cached, base + lane, 32, hi);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * 32 + lane;
+      const uint32_t k = kk[u] & mask;
+      const bool gt = i < hi && k > prefix;
+      const bool eq = i < hi && k == prefix;
+      const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+      const int my_eq_rank = pos_eq + __popc(beq & below);
+      const int slot = pos_gt + __popc(bgt & below) + min(my_eq_rank, need);
+      if ((gt || (eq && my_eq_rank < need)) && slot < K) out[slot] = i;
+      pos_gt += __popc(bgt);
+      pos_eq += __popc(beq);
+    }
   }
 }
 
@@ -454,16 +533,13 @@ cudaError_t launch_topk(const IndexerArgs& a, int64_t r0, int64_t r1, cudaStream
   const int64_t rows = r1 - r0;
   const bool wide = a.P_cap > 4096 && rows < 4 * 148;
   const bool uncached = a.P_cap > 4096 && !wide;
-  const size_t smem = uncached ? (size_t)kTopkCand * sizeof(uint64_t)
+  const size_t smem = uncached ? (size_t)kTopkListBytes
                                : (size_t)(a.P_cap < kTopkSmemKeys ? a.P_cap : kTopkSmemKeys) * sizeof(uint32_t);
   const int cache_keys = uncached ? 0 : (int)(smem / sizeof(uint32_t));
-  cudaError_t e = wide ? cudaFuncSetAttribute(topk_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                       : cudaFuncSetAttribute(topk_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  void (*kern)(IndexerArgs, int64_t, int) = wide ? topk_kernel<1024> : topk_kernel<256>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if (wide)
-    topk_kernel<1024><<<(unsigned)(r1 - r0), 1024, smem, st>>>(a, r0, cache_keys);
-  else
-    topk_kernel<256><<<(unsigned)(r1 - r0), 256, smem, st>>>(a, r0, cache_keys);
+  kern<<<(unsigned)(r1 - r0), wide ? 1024 : 256, smem, st>>>(a, r0, cache_keys);
   note_launch();
   return cudaGetLastError();
 }

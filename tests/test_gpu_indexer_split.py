@@ -109,19 +109,31 @@ def test_topk_select_bit_exact(lib, P_cap, topk):
 @pytest.mark.parametrize("topk", [512, 2048])
 def test_topk_select_many_long_rows_bit_exact(lib, topk):
     """Hundreds of rows longer than 4096 entries take the path that re-reads each row from its
-    scores (256 threads per row, several rows per SM): there the keys of the threshold digit
-    are kept in shared memory when there are at most 2048 of them, and the row is read three
-    times.  Rows of narrow-range distinct scores take that path; tie-heavy rows (thousands of
-    keys in one digit) the general one.  Every row against the oracle's ranking."""
+    scores (256 threads per row, several rows per SM): each warp lists the entries of its
+    segment at or above the threshold digit, and the rest of the selection goes over the lists.
+    Row kinds: tie-heavy (small integers: lists of tied keys; an all-equal row, whose lists
+    overflow and whose threshold digit holds one value); narrow-range distinct scores (every
+    key in one digit: the lists overflow and the row is read again digit by digit); the
+    one-head indexer's shape, w * ReLU(x) with half of the entries an exact +0 or -0 (w > 0:
+    short lists; w < 0: the kept entries are the first exact zeros); and decreasing scores,
+    whose kept entries all sit in the first warps' segments.  Every row against the oracle's
+    ranking."""
     abi, harness = lib
     P_cap, Sq = 9000, 700
     rng = np.random.default_rng(20261203 + topk)
     q_index = rng.integers(0, P_cap, size=(1, Sq)).astype(np.int32)
-    q_index[0, :4] = [P_cap - 1, topk - 1, topk, 4096]
+    q_index[0, :6] = [P_cap - 1, topk - 1, topk, 4096, P_cap - 1, P_cap - 1]
     sc = _tie_heavy_scores(rng, Sq, P_cap)
-    spread = rng.random(Sq) < 0.5
-    spread[:2] = [False, True]
+    kind = rng.integers(0, 4, size=Sq)
+    kind[:6] = [0, 1, 0, 0, 2, 3]
+    spread = kind == 1
     sc[spread] = (1.0 + rng.random((int(spread.sum()), P_cap)) * 1e-3).astype(np.float32)
+    relu = kind == 2
+    x = rng.standard_normal((int(relu.sum()), P_cap)).astype(np.float32)
+    wsign = np.where(rng.random((int(relu.sum()), 1)) < 0.5, np.float32(-1.5), np.float32(1.5))
+    sc[relu] = (wsign * np.maximum(x, np.float32(0.0))).astype(np.float32)  # -1.5 * 0 = -0
+    dec = kind == 3
+    sc[dec] = (np.float32(1e4) - np.arange(P_cap, dtype=np.float32))[None, :]
     w = synth.WORKLOADS["csa_decode_bf16"].replace(B=1, Sq=Sq, S=P_cap, m=1, P_cap=P_cap, topk=topk)
     params = harness.params_for(w)
     idx = torch.full((1, Sq, topk), -7, dtype=torch.int32, device="cuda")
