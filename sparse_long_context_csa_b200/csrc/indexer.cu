@@ -147,6 +147,31 @@ __device__ __forceinline__ void row_keys8(uint32_t (&k)[8], const uint32_t* keys
   }
 }
 
+// The keys of the eight consecutive entries e0 .. e0 + 7 (e0 a multiple of 8), 0 at or past
+// `end`: two 16-byte loads when `vec` (every row starts on 16 bytes and holds a multiple of 4
+// entries, so a vector that starts below `end` stays inside the row), else eight 4-byte ones.
+__device__ __forceinline__ void row_run8(uint32_t (&k)[8], const float* sc, bool vec, int e0, int end) {
+  float v[8];
+  if (vec) {
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 x = e0 < end ? *reinterpret_cast<const float4*>(sc + e0) : z;
+    const float4 y = e0 + 4 < end ? *reinterpret_cast<const float4*>(sc + e0 + 4) : z;
+    v[0] = x.x;
+    v[1] = x.y;
+    v[2] = x.z;
+    v[3] = x.w;
+    v[4] = y.x;
+    v[5] = y.y;
+    v[6] = y.z;
+    v[7] = y.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = e0 + j < end ? sc[e0 + j] : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) k[j] = order_key(v[j]);
+}
+
 // Finds the digit holding the need-th largest key of a histogram (digits scanned from the
 // top): *bin = that digit, *rest = how many keys of it are still needed, *cnt = its count.
 // Thread t owns the descending run of digits [top - BPT + 1, top], top = kTopkBins-1-t*BPT.
@@ -237,17 +262,18 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   }
   const float* sc = a.scores + (int64_t)blockIdx.x * a.P_cap;
   const bool cached = vis <= cache_keys;  // keys kept in shared memory
+  const bool vec = (a.P_cap & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
   for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
   __syncthreads();
-  for (int base = tid; base < vis; base += NT * 8) {
+  // each thread takes runs of eight consecutive entries
+  for (int e0 = tid * 8; e0 < vis; e0 += NT * 8) {
     uint32_t kk[8];
-    row_keys8(kk, keys, sc, false, base, NT, vis);
+    row_run8(kk, sc, vec, e0, vis);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = base + u * NT;
-      if (j < vis) {
-        if (cached) keys[j] = kk[u];
-        atomicAdd(&hist[kk[u] >> 20], 1u);
+    for (int j = 0; j < 8; ++j) {
+      if (e0 + j < vis) {
+        if (cached) keys[e0 + j] = kk[j];
+        atomicAdd(&hist[kk[j] >> 20], 1u);
       }
     }
   }
@@ -255,7 +281,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
   uint32_t prefix = (uint32_t)s_bin << 20, mask = 0xFFF00000u;
   int need = s_rest;
-  const int seg = (vis + kWarps - 1) / kWarps;
+  const int seg = ((vis + kWarps - 1) / kWarps + 7) & ~7;  // warp segments start on 8 entries
   const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
   int n_gt = 0, n_eq = 0;  // this warp segment's keys above / equal to the final prefix
   bool counted = false, listed = false;
@@ -271,27 +297,41 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
       s_kmax = 0u;
     }
     __syncthreads();
+    // lane l takes the run of eight entries base + 8l .. base + 8l + 7; a scan of the lanes'
+    // counts places each run's listed entries
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int base = lo; base < hi; base += 32 * 8) {
+      const int e0 = base + lane * 8;
       uint32_t kk[8];
-      row_keys8(kk, keys, sc, false, base + lane, 32, hi);
+      row_run8(kk, sc, vec, e0, hi);
+      uint32_t selm = 0u, digm = 0u;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = base + u * 32 + lane;
-        const uint32_t dg = kk[u] >> 20;
-        const bool sel = i < hi && dg >= b1;
-        const unsigned bs = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-          const int pos = len + __popc(bs & below);
-          if (pos < kCap) list[pos] = (uint32_t)i | (dg == b1 ? kListDigit : 0u);
-          if (track && dg == b1) {
-            n_eq += 1;
-            kmin = min(kmin, kk[u]);
-            kmax = max(kmax, kk[u]);
-          }
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t dg = kk[j] >> 20;
+        const bool sel = e0 + j < hi && dg >= b1;
+        selm |= (uint32_t)sel << j;
+        digm |= (uint32_t)(dg == b1) << j;
+        if (track && sel && dg == b1) {
+          n_eq += 1;
+          kmin = min(kmin, kk[j]);
+          kmax = max(kmax, kk[j]);
         }
-        len += __popc(bs);
       }
+      const int c = __popc(selm);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (len < kCap) {
+        int pos = len + incl - c;
+        for (uint32_t m = selm; m != 0u; m &= m - 1u, ++pos) {
+          const int j = __ffs(m) - 1;
+          if (pos < kCap) list[pos] = (uint32_t)(e0 + j) | ((digm >> j) & 1u ? kListDigit : 0u);
+        }
+      }
+      len += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0 && len > kCap) s_over = 1;
     if (track) {
