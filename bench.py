@@ -166,15 +166,16 @@ def roofline_of(name, flops, nbytes, ms, peaks, peak_src, kind="burst"):
 # the kernel definition, and the headers it includes): once any of it changes, traffic reads
 # null until the kernel is captured again.  Values: (source segments, sha256, bytes per launch).
 _ATTN_SOURCE = (("attn_tc.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("common.cuh", None),
-                ("internal.h", None))
+                ("internal.h", None), ("select.cuh", None))
 _INDEXER_SOURCE = (("indexer_tc.cu", "\n}  // namespace\n\nbool indexer_tc_supported"), ("tc_ptx.cuh", None),
                    ("common.cuh", None), ("internal.h", None), ("select.cuh", None))
 _OUT_PROJ_SOURCE = (("out_proj.cu", "\ntypedef CUresult (*EncodeTiledFn)"), ("tc_ptx.cuh", None), ("internal.h", None))
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the CSA prefill step (B=1, S=8192, H=64, D=dv=512, top-512,
     # window 128; the kernel selects each query's index list from its score row):
-    # dram__bytes_read.sum 579.6 MB + dram__bytes_write.sum 511.7 MB.
-    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "a54fe13d9175d88c22216ab380fc2c4f3bef9006147a65baa85af78a9690ecd7", 1091308544),
+    # dram__bytes_read.sum 579.6 MB + dram__bytes_write.sum 511.7 MB.  (Re-keyed when the hash
+    # took in select.cuh, which attn_tc.cu includes; it has not changed since the capture.)
+    ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "c39ebe7dad0102f834d73fa380b0cf0c41b674c81b356b8a5dadc60a1abe8bde", 1091308544),
     # ncu --set full, one launch of the CSA decode step (64 queries, pool 32768, top-2048): the fused
     # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.5 MB.  (Re-keyed
     # when internal.h gained the attention's score-row fields; nothing this kernel compiles changed.)
