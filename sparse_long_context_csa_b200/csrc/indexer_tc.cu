@@ -90,6 +90,7 @@ struct IdxMisc {
   uint64_t full[kStages], empty[kStages], tfull[2], tempty[2];
   uint32_t tmem_base;
   int maxvis;
+  int minvis;  // the least visible-entry count of the group's rows (0 when a row is past the chunk)
   int abort_flag;
   int sel_last;  // fused selection: this CTA merges the splits of its query
   int vis[256];
@@ -100,8 +101,9 @@ static_assert(offsetof(IdxMisc, w) % 16 == 0, "weights are read as float4");
 
 // Scores of one 32-column chunk of the accumulator (columns c .. c+31, column = q * NI + h)
 // for the entry of this thread: whole queries for NI <= 32; for NI = 64 two chunks make one
-// query (the first leaves its partial sum in `carry`).
-template <int NI>
+// query (the first leaves its partial sum in `carry`).  kFull: the tile's entries are visible
+// to every query of the group, so no score is masked.
+template <int NI, bool kFull>
 __device__ __forceinline__ void score_chunk(const float (&acc)[32], int c, const float* wsm, const int* vis, int nq,
                                             int w, float* sbase, int64_t P_cap, float& carry) {
   float wv[32];
@@ -114,13 +116,15 @@ __device__ __forceinline__ void score_chunk(const float (&acc)[32], int c, const
     wv[4 * k + 3] = v.w;
   }
   if constexpr (NI <= 32) {
+    float* out = sbase + (int64_t)(c / NI) * P_cap;
 #pragma unroll
     for (int qq = 0; qq < 32 / NI; ++qq) {
       float sc = 0.f;
 #pragma unroll
       for (int h = 0; h < NI; ++h) sc = fmaf(wv[qq * NI + h], fmaxf(acc[qq * NI + h], 0.f), sc);
       const int q = c / NI + qq;
-      if (q < nq && w < vis[q]) sbase[(int64_t)q * P_cap] = sc;
+      if (kFull || (q < nq && w < vis[q])) *out = sc;
+      out += P_cap;
     }
   } else {
     float s0 = 0.f, s1 = 0.f;
@@ -133,7 +137,7 @@ __device__ __forceinline__ void score_chunk(const float (&acc)[32], int c, const
       carry = s0 + s1;
     } else {
       const int q = c / 64;
-      if (q < nq && w < vis[q]) sbase[(int64_t)q * P_cap] = carry + s0 + s1;
+      if (kFull || (q < nq && w < vis[q])) sbase[(int64_t)q * P_cap] = carry + s0 + s1;
     }
   }
 }
@@ -141,12 +145,15 @@ __device__ __forceinline__ void score_chunk(const float (&acc)[32], int c, const
 // The epilogue of one tile for this thread's chunks [k_lo, k_hi) of 32 columns.
 template <int NI>
 __device__ __forceinline__ void score_tile(uint32_t taddr, int k_lo, int k_hi, const float* wsm, const int* vis,
-                                           int nq, int w, float* sbase, int64_t P_cap) {
+                                           int nq, int w, float* sbase, int64_t P_cap, bool full) {
   float carry = 0.f;
   for (int k = k_lo; k < k_hi; ++k) {
     float acc[32];
     tc::tmem_ld_x32(taddr + 32 * k, acc);
-    score_chunk<NI>(acc, 32 * k, wsm, vis, nq, w, sbase, P_cap, carry);
+    if (full)
+      score_chunk<NI, true>(acc, 32 * k, wsm, vis, nq, w, sbase, P_cap, carry);
+    else
+      score_chunk<NI, false>(acc, 32 * k, wsm, vis, nq, w, sbase, P_cap, carry);
   }
 }
 
@@ -191,6 +198,7 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
       tc::mbar_init(&ms->tempty[i], kEpilogue);
     }
     ms->maxvis = 0;
+    ms->minvis = 0x7fffffff;
     ms->abort_flag = 0;
     tc::mbar_fence_init();
   }
@@ -206,6 +214,7 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     }
     ms->vis[q] = v;
     atomicMax(&ms->maxvis, v);
+    atomicMin(&ms->minvis, v);
   }
   for (int i = tid; i < 256 + 32; i += kThreads) ms->w[i] = (i < QB * nI && (i / nI) < nq) ? a.wI[rbase * nI + i] : 0.f;
   __syncthreads();
@@ -355,17 +364,20 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
               a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
           }
         }
-      } else {
+      } else if constexpr (!kSelect) {  // the fused selection has one query of <= 16 heads: small
         float* sbase = a.scores + (rbase - P.row0) * a.P_cap + w;
         const uint32_t taddr = tmem + tb * Npad + lane_off;
+        // every entry of the tile visible to every query of the group (all but the causal
+        // diagonal of prefill): no per-score mask
+        const bool full = (t_lo + i + 1) * kTileE <= ms->minvis;
         switch (nI) {
-          case 1: score_tile<1>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          case 2: score_tile<2>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          case 4: score_tile<4>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          case 8: score_tile<8>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          case 16: score_tile<16>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          case 32: score_tile<32>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
-          default: score_tile<64>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap); break;
+          case 1: score_tile<1>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          case 2: score_tile<2>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          case 4: score_tile<4>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          case 8: score_tile<8>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          case 16: score_tile<16>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          case 32: score_tile<32>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
+          default: score_tile<64>(taddr, k_lo, k_hi, ms->w, ms->vis, nq, w, sbase, a.P_cap, full); break;
         }
       }
       tc::tc_fence_before();
