@@ -223,6 +223,53 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* 
   __syncthreads();
 }
 
+// One warp lists, in entry order, the entries e of [lo, hi) whose key's top digit is at least
+// b1: list[p] = e, with kListDigit set when the digit is b1 (entries past kCap are counted,
+// not stored).  Lane l takes the run of eight entries base + 8l .. base + 8l + 7 and a scan of
+// the lanes' counts places each run's entries.  With `track`, each lane also counts its keys
+// of digit b1 and keeps their least and greatest.  Returns the segment's number of listed
+// entries (the same in every lane).
+template <int kCap>
+__device__ __forceinline__ int list_segment(const float* sc, bool vec, int lo, int hi, uint32_t b1, bool track,
+                                            uint32_t* list, int& n_eq, uint32_t& kmin, uint32_t& kmax) {
+  const int lane = threadIdx.x & 31;
+  int len = 0;
+  for (int base = lo; base < hi; base += 32 * 8) {
+    const int e0 = base + lane * 8;
+    uint32_t kk[8];
+    row_run8(kk, sc, vec, e0, hi);
+    uint32_t selm = 0u, digm = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t dg = kk[j] >> 20;
+      const bool sel = e0 + j < hi && dg >= b1;
+      selm |= (uint32_t)sel << j;
+      digm |= (uint32_t)(dg == b1) << j;
+      if (track && sel && dg == b1) {
+        n_eq += 1;
+        kmin = min(kmin, kk[j]);
+        kmax = max(kmax, kk[j]);
+      }
+    }
+    const int c = __popc(selm);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (len < kCap) {
+      int pos = len + incl - c;
+      for (uint32_t m = selm; m != 0u; m &= m - 1u, ++pos) {
+        const int j = __ffs(m) - 1;
+        if (pos < kCap) list[pos] = (uint32_t)(e0 + j) | ((digm >> j) & 1u ? kListDigit : 0u);
+      }
+    }
+    len += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return len;
+}
+
 // Per-query top-k by radix select over order-preserving keys: a 12-bit digit histogram
 // while the row is loaded, then 12 and 8 more bits over the keys that still match the
 // selected prefix (skipped once the threshold digit holds exactly the keys still needed).
@@ -235,13 +282,15 @@ __device__ __forceinline__ void find_digit(const uint32_t* hist, int need, int* 
 // of shared memory sends the row to the passes over the whole row; when the threshold digit
 // holds one value only (a long run of equal scores, such as the exact zeros that ReLU leaves
 // in a one-head indexer), that value is the whole prefix and the counts come from the same
-// pass.
+// pass.  A row of at least 4 topk entries first takes its threshold digit from an eighth of
+// its entries instead of the full histogram (see below), so it reads its scores about 1.1
+// times when that works.
 template <int NT>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs a, int64_t row0, int cache_keys) {
   extern __shared__ __align__(16) uint32_t keys[];  // the row's keys (cached rows) or the warps' lists
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int wsum[NT / 32];
-  __shared__ int s_bin, s_rest, s_cnt, s_over;
+  __shared__ int s_bin, s_rest, s_cnt, s_over, s_len, s_eq;
   __shared__ uint32_t s_kmin, s_kmax;
   __shared__ int wcnt_gt[NT / 32], wcnt_eq[NT / 32];
   constexpr int kWarps = NT / 32;
@@ -262,101 +311,146 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
   }
   const float* sc = a.scores + (int64_t)blockIdx.x * a.P_cap;
   const bool cached = vis <= cache_keys;  // keys kept in shared memory
+  const bool uncached = !cached && cache_keys == 0;
   const bool vec = (a.P_cap & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
-  for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
-  __syncthreads();
-  // each thread takes runs of eight consecutive entries
-  for (int e0 = tid * 8; e0 < vis; e0 += NT * 8) {
-    uint32_t kk[8];
-    row_run8(kk, sc, vec, e0, vis);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (e0 + j < vis) {
-        if (cached) keys[e0 + j] = kk[j];
-        atomicAdd(&hist[kk[j] >> 20], 1u);
-      }
-    }
-  }
-  __syncthreads();
-  find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
-  uint32_t prefix = (uint32_t)s_bin << 20, mask = 0xFFF00000u;
-  int need = s_rest;
   const int seg = ((vis + kWarps - 1) / kWarps + 7) & ~7;  // warp segments start on 8 entries
   const int lo = min(vis, warp * seg), hi = min(vis, lo + seg);
-  int n_gt = 0, n_eq = 0;  // this warp segment's keys above / equal to the final prefix
-  bool counted = false, listed = false;
-  int len = 0;  // entries at or above the threshold digit in this warp's segment
   uint32_t* list = keys + warp * kCap;
-  if (!cached && cache_keys == 0) {
-    const uint32_t b1 = (uint32_t)s_bin;
-    // a list can outgrow its share only when the entries to list outnumber one share
-    const bool track = K - need + s_cnt > kCap;
+  uint32_t prefix = 0u, mask = 0xFFF00000u;
+  int need = 0;
+  int n_gt = 0, n_eq = 0;  // this warp segment's keys above / equal to the final prefix
+  int len = 0;             // entries of this warp's segment in its list
+  bool counted = false, listed = false;
+  bool allcand = false;  // the lists hold candidates of a sampled threshold: every key is compared
+
+  // A long uncached row first takes its threshold digit from a sample (the first 32 entries of
+  // every 256), placed so that about 5/4 topk entries of the row lie at or above it, and lists
+  // them.  The selection is then exact over the lists when they hold at least topk entries and
+  // fit; when they overflow only because the threshold digit is one long run of a value that
+  // holds the topk-th key, the counts are done as below; otherwise the row starts again on the
+  // general path.
+  if (uncached && vis >= 4 * K) {
+    for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
     if (tid == 0) {
       s_over = 0;
+      s_len = 0;
+      s_eq = 0;
       s_kmin = 0xFFFFFFFFu;
       s_kmax = 0u;
     }
     __syncthreads();
-    // lane l takes the run of eight entries base + 8l .. base + 8l + 7; a scan of the lanes'
-    // counts places each run's listed entries
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int base = lo; base < hi; base += 32 * 8) {
-      const int e0 = base + lane * 8;
-      uint32_t kk[8];
-      row_run8(kk, sc, vec, e0, hi);
-      uint32_t selm = 0u, digm = 0u;
+    for (int c0 = warp; c0 * 256 < vis; c0 += kWarps * 8) {
+      float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t dg = kk[j] >> 20;
-        const bool sel = e0 + j < hi && dg >= b1;
-        selm |= (uint32_t)sel << j;
-        digm |= (uint32_t)(dg == b1) << j;
-        if (track && sel && dg == b1) {
-          n_eq += 1;
-          kmin = min(kmin, kk[j]);
-          kmax = max(kmax, kk[j]);
-        }
+      for (int u = 0; u < 8; ++u) {
+        const int e = (c0 + u * kWarps) * 256 + lane;
+        v[u] = e < vis ? sc[e] : 0.f;
       }
-      const int c = __popc(selm);
-      int incl = c;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      if (len < kCap) {
-        int pos = len + incl - c;
-        for (uint32_t m = selm; m != 0u; m &= m - 1u, ++pos) {
-          const int j = __ffs(m) - 1;
-          if (pos < kCap) list[pos] = (uint32_t)(e0 + j) | ((digm >> j) & 1u ? kListDigit : 0u);
-        }
-      }
-      len += __shfl_sync(0xffffffffu, incl, 31);
+      for (int u = 0; u < 8; ++u)
+        if ((c0 + u * kWarps) * 256 + lane < vis) atomicAdd(&hist[order_key(v[u]) >> 20], 1u);
     }
-    if (lane == 0 && len > kCap) s_over = 1;
-    if (track) {
-      kmin = __reduce_min_sync(0xffffffffu, kmin);
-      kmax = __reduce_max_sync(0xffffffffu, kmax);
-      n_eq = __reduce_add_sync(0xffffffffu, n_eq);
-      if (lane == 0 && kmin <= kmax) {
+    __syncthreads();
+    const int ns = (vis >> 8) * 32 + min(32, vis & 255);  // sampled entries
+    const int ks = min(ns, (int)((int64_t)K * ns * 5 / (4 * (int64_t)vis)) + 32);
+    find_digit<NT>(hist, ks, wsum, &s_bin, &s_rest, &s_cnt);
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    int eqc = 0;
+    len = list_segment<kCap>(sc, vec, lo, hi, (uint32_t)s_bin, true, list, eqc, kmin, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    eqc = __reduce_add_sync(0xffffffffu, eqc);
+    if (lane == 0) {
+      if (len > kCap) s_over = 1;
+      atomicAdd(&s_len, len);
+      atomicAdd(&s_eq, eqc);
+      if (kmin <= kmax) {
         atomicMin(&s_kmin, kmin);
         atomicMax(&s_kmax, kmax);
       }
     }
     __syncthreads();
-    listed = s_over == 0;
-    if (!listed && s_cnt != need && s_kmin == s_kmax) {
-      // the threshold digit holds one value: it is the whole prefix, and the counts are done
+    const int tot = s_len, tot_gt = s_len - s_eq;
+    if (s_over == 0 && tot >= K) {
+      listed = true;
+      allcand = true;
+    } else if (s_over != 0 && tot_gt < K && tot >= K && s_kmin == s_kmax) {
       prefix = s_kmin;
       mask = 0xFFFFFFFFu;
-      n_gt = len - n_eq;
+      need = K - tot_gt;
+      n_gt = len - eqc;
+      n_eq = eqc;
       counted = true;
-    } else {
-      n_eq = 0;
+    }
+    __syncthreads();  // every thread has read the shared words before the general path resets them
+  }
+  if (!listed && !counted) {
+    for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
+    __syncthreads();
+    // each thread takes runs of eight consecutive entries
+    for (int e0 = tid * 8; e0 < vis; e0 += NT * 8) {
+      uint32_t kk[8];
+      row_run8(kk, sc, vec, e0, vis);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (e0 + j < vis) {
+          if (cached) keys[e0 + j] = kk[j];
+          atomicAdd(&hist[kk[j] >> 20], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
+    prefix = (uint32_t)s_bin << 20;
+    need = s_rest;
+    len = 0;
+    if (uncached) {
+      // a list can outgrow its share only when the entries to list outnumber one share
+      const bool track = K - need + s_cnt > kCap;
+      if (tid == 0) {
+        s_over = 0;
+        s_kmin = 0xFFFFFFFFu;
+        s_kmax = 0u;
+      }
+      __syncthreads();
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+      len = list_segment<kCap>(sc, vec, lo, hi, (uint32_t)s_bin, track, list, n_eq, kmin, kmax);
+      if (lane == 0 && len > kCap) s_over = 1;
+      if (track) {
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+        if (lane == 0 && kmin <= kmax) {
+          atomicMin(&s_kmin, kmin);
+          atomicMax(&s_kmax, kmax);
+        }
+      }
+      __syncthreads();
+      listed = s_over == 0;
+      if (!listed && s_cnt != need && s_kmin == s_kmax) {
+        // the threshold digit holds one value: it is the whole prefix, and the counts are done
+        prefix = s_kmin;
+        mask = 0xFFFFFFFFu;
+        n_gt = len - n_eq;
+        counted = true;
+      } else {
+        n_eq = 0;
+      }
     }
   }
   if (listed) {
-    // the remaining 12 and 8 bits over the listed threshold-digit entries
+    if (allcand) {
+      // the top digit over every listed entry
+      for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0u;
+      __syncthreads();
+      for (int p = lane; p < len; p += 32) atomicAdd(&hist[order_key(sc[list[p] & ~kListDigit]) >> 20], 1u);
+      __syncthreads();
+      find_digit<NT>(hist, K, wsum, &s_bin, &s_rest, &s_cnt);
+      prefix = (uint32_t)s_bin << 20;
+      need = s_rest;
+    }
+    // the remaining 12 and 8 bits over the listed entries of the threshold digit (every
+    // listed entry after a sampled threshold)
     for (int pass = 1; pass < 3 && s_cnt != need; ++pass) {
       const int shift = pass == 1 ? 8 : 0;
       const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
@@ -364,7 +458,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
       __syncthreads();
       for (int p = lane; p < len; p += 32) {
         const uint32_t e = list[p];
-        if (e & kListDigit) {
+        if (allcand || (e & kListDigit)) {
           const uint32_t k = order_key(sc[e & ~kListDigit]);
           if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
         }
@@ -379,7 +473,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
     // threshold digit are above it)
     for (int p = lane; p < len; p += 32) {
       const uint32_t e = list[p];
-      if (e & kListDigit) {
+      if (allcand || (e & kListDigit)) {
         const uint32_t k = order_key(sc[e & ~kListDigit]) & mask;
         n_gt += k > prefix;
         n_eq += k == prefix;
@@ -452,7 +546,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 6 : 1) topk_kernel(IndexerArgs
     for (int base = 0; base < len; base += 32) {
       const int p = base + lane;
       const uint32_t e = p < len ? list[p] : 0u;
-      const bool dig = (e & kListDigit) != 0u;
+      const bool dig = allcand || (e & kListDigit) != 0u;
       const uint32_t k = dig ? order_key(sc[e & ~kListDigit]) & mask : 0u;
       const bool gt = p < len && (!dig || k > prefix);
       const bool eq = p < len && dig && k == prefix;

@@ -115,17 +115,20 @@ def test_topk_select_many_long_rows_bit_exact(lib, topk):
     overflow and whose threshold digit holds one value); narrow-range distinct scores (every
     key in one digit: the lists overflow and the row is read again digit by digit); the
     one-head indexer's shape, w * ReLU(x) with half of the entries an exact +0 or -0 (w > 0:
-    short lists; w < 0: the kept entries are the first exact zeros); and decreasing scores,
-    whose kept entries all sit in the first warps' segments.  Every row against the oracle's
-    ranking."""
+    short lists; w < 0: the kept entries are the first exact zeros); decreasing scores, whose
+    kept entries all sit in the first warps' segments; and two kinds that defeat a threshold
+    taken from a sample of the first 32 entries of every 256 (peaks only where the sample does
+    not look: too many entries at or above it; peaks only where it looks: too few), so those
+    rows start again on the general path.  Every row against the oracle's ranking."""
     abi, harness = lib
     P_cap, Sq = 9000, 700
     rng = np.random.default_rng(20261203 + topk)
     q_index = rng.integers(0, P_cap, size=(1, Sq)).astype(np.int32)
     q_index[0, :6] = [P_cap - 1, topk - 1, topk, 4096, P_cap - 1, P_cap - 1]
     sc = _tie_heavy_scores(rng, Sq, P_cap)
-    kind = rng.integers(0, 4, size=Sq)
-    kind[:6] = [0, 1, 0, 0, 2, 3]
+    kind = rng.integers(0, 6, size=Sq)
+    kind[:8] = [0, 1, 0, 0, 2, 3, 4, 5]
+    q_index[0, 6:8] = P_cap - 1
     spread = kind == 1
     sc[spread] = (1.0 + rng.random((int(spread.sum()), P_cap)) * 1e-3).astype(np.float32)
     relu = kind == 2
@@ -134,6 +137,12 @@ def test_topk_select_many_long_rows_bit_exact(lib, topk):
     sc[relu] = (wsign * np.maximum(x, np.float32(0.0))).astype(np.float32)  # -1.5 * 0 = -0
     dec = kind == 3
     sc[dec] = (np.float32(1e4) - np.arange(P_cap, dtype=np.float32))[None, :]
+    in_sample = (np.arange(P_cap) % 256) < 32
+    for k, where in ((4, ~in_sample & (np.arange(P_cap) % 5 == 0)), (5, in_sample)):
+        rows = kind == k
+        base = (rng.standard_normal((int(rows.sum()), P_cap)) * 0.01).astype(np.float32)
+        peak = (10.0 + rng.standard_normal((int(rows.sum()), P_cap))).astype(np.float32)
+        sc[rows] = np.where(where[None, :], peak, base)
     w = synth.WORKLOADS["csa_decode_bf16"].replace(B=1, Sq=Sq, S=P_cap, m=1, P_cap=P_cap, topk=topk)
     params = harness.params_for(w)
     idx = torch.full((1, Sq, topk), -7, dtype=torch.int32, device="cuda")
