@@ -71,7 +71,7 @@ struct IdxTcParams {
 };
 
 struct IdxSmem {
-  uint32_t a, b, misc, sel, total;
+  uint32_t a, b, misc, sel, hist, total;
 };
 
 // sel_entries: scores kept in shared memory by the fused selection (0: none)
@@ -82,7 +82,8 @@ __host__ __device__ inline IdxSmem idx_smem_layout(int cI, int Npad, int sel_ent
   s.b = s.a + kStages * nch * 16384;                // nch x Npad x 128 B
   s.misc = s.b + nch * ((Npad * 128 + 1023) / 1024) * 1024;
   s.sel = s.misc + 4096;                            // sel_entries fp32 scores
-  s.total = s.sel + (uint32_t)sel_entries * 4;
+  s.hist = s.sel + (uint32_t)sel_entries * 4;       // their top-digit histogram (kSelBins words)
+  s.total = s.hist + (sel_entries > 0 ? kSelBins * 4 : 0);
   return s;
 }
 
@@ -163,6 +164,111 @@ constexpr int kSelKeysOffset = 20480;      // merge: candidate keys after the hi
 constexpr int64_t kSelMinEntries = int64_t(1) << 20;  // scored entries per launch below which it is not used
 
 __device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 3, 512;" ::: "memory"); }
+
+// The split's top-K candidates (n > K scores in shared memory) from the histogram of their
+// top 12-bit digits, built by the epilogue while it scored: the digit holding the K-th key,
+// then one pass in which each warp lists, in entry order, the entries of its segment at or
+// above that digit (bit 31 marks those in it), then the remaining 12 and 8 bits, the counts
+// and the ordered write over the lists.  Writes the same candidates, in the same order, as
+// select_topk.  Returns false, having written nothing, when a list outgrows its `cap`
+// entries (the caller then runs select_topk).  Every thread of the selection calls it.
+__device__ __forceinline__ bool split_select_listed(const float* ssc, int n, int K, int w0, const uint32_t* shist,
+                                                    uint32_t* hist, SelShared<kSelThreads>* sh, uint32_t* lists,
+                                                    int cap, uint64_t* cand) {
+  constexpr int kWarps = kSelThreads / 32;
+  constexpr uint32_t kIn = 0x80000000u;  // list flag: the key is in the threshold digit
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned below = (1u << lane) - 1u;
+  int* over = reinterpret_cast<int*>(hist + kSelBins - 1);  // a histogram word, free here
+  select_digit<kSelThreads>(shist, K, tid, sh, sel_sync);
+  const uint32_t b1 = (uint32_t)sh->bin;
+  int need = sh->rest, cnt = sh->cnt;
+  if (tid == 0) *over = 0;
+  sel_sync();
+  uint32_t* lst = lists + warp * cap;
+  const int seg = (n + kWarps - 1) / kWarps;
+  const int lo = min(n, warp * seg), hi = min(n, lo + seg);
+  int len = 0;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t dg = i < hi ? order_key(ssc[i]) >> 20 : 0u;
+    const bool sel = i < hi && dg >= b1;
+    const unsigned bs = __ballot_sync(0xffffffffu, sel);
+    const int pos = len + __popc(bs & below);
+    if (sel && pos < cap) lst[pos] = (uint32_t)i | (dg == b1 ? kIn : 0u);
+    len += __popc(bs);
+  }
+  if (lane == 0 && len > cap) atomicOr(over, 1);
+  sel_sync();
+  if (*over) {
+    sel_sync();  // every thread has read the flag before select_topk reuses the histogram
+    return false;
+  }
+  uint32_t prefix = b1 << 20, mask = 0xFFF00000u;
+  for (int pass = 1; pass < 3 && cnt != need; ++pass) {
+    const int shift = pass == 1 ? 8 : 0;
+    const uint32_t dmask = pass == 1 ? 0xFFFu : 0xFFu;
+    for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0u;
+    sel_sync();
+    for (int p = lane; p < len; p += 32) {
+      const uint32_t e = lst[p];
+      if (e & kIn) {
+        const uint32_t k = order_key(ssc[e & ~kIn]);
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+      }
+    }
+    sel_sync();
+    select_digit<kSelThreads>(hist, need, tid, sh, sel_sync);
+    prefix |= (uint32_t)sh->bin << shift;
+    mask |= dmask << shift;
+    need = sh->rest;
+    cnt = sh->cnt;
+  }
+  // this segment's listed keys above / equal to the final prefix (entries outside the
+  // threshold digit are above it), a scan over warps, then the ordered write
+  int n_gt = 0, n_eq = 0;
+  for (int p = lane; p < len; p += 32) {
+    const uint32_t e = lst[p];
+    if (e & kIn) {
+      const uint32_t k = order_key(ssc[e & ~kIn]) & mask;
+      n_gt += k > prefix;
+      n_eq += k == prefix;
+    } else {
+      n_gt += 1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+  }
+  if (lane == 0) {
+    sh->wcnt_gt[warp] = n_gt;
+    sh->wcnt_eq[warp] = n_eq;
+  }
+  sel_sync();
+  int pos_gt = 0, pos_eq = 0;
+  for (int w = 0; w < warp; ++w) {
+    pos_gt += sh->wcnt_gt[w];
+    pos_eq += sh->wcnt_eq[w];
+  }
+  for (int base = 0; base < len; base += 32) {
+    const int p = base + lane;
+    const uint32_t e = p < len ? lst[p] : 0u;
+    const uint32_t key = p < len ? order_key(ssc[e & ~kIn]) : 0u;
+    const bool gt = p < len && (!(e & kIn) || (key & mask) > prefix);
+    const bool eq = p < len && (e & kIn) && (key & mask) == prefix;
+    const unsigned bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+    const int my_eq_rank = pos_eq + __popc(beq & below);
+    const int slot = pos_gt + __popc(bgt & below) + min(my_eq_rank, need);
+    if ((gt || (eq && my_eq_rank < need)) && slot < K)
+      cand[slot] = ((uint64_t)key << 32) | (uint32_t)(w0 + (int)(e & ~kIn));
+    pos_gt += __popc(bgt);
+    pos_eq += __popc(beq);
+  }
+  sel_sync();
+  return true;
+}
 
 template <bool kSelect>
 __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P) {
@@ -253,6 +359,9 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   }
+  uint32_t* shist = reinterpret_cast<uint32_t*>(smem + L.hist);  // fused selection: top digits of ssc
+  if constexpr (kSelect)
+    for (int i = tid; i < kSelBins; i += blockDim.x) shist[i] = 0u;
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
@@ -358,9 +467,10 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
             float sc = 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) sc = fmaf(qcol[j] == q ? wsm[j] : 0.f, fmaxf(acc[j], 0.f), sc);
-            if (kSelect)
+            if (kSelect) {
               ssc[i * kTileE + e] = sc;  // one query per group; entries past vis are never read
-            else if (w < ms->vis[q])
+              if (w < ms->vis[q]) atomicAdd(&shist[order_key(sc) >> 20], 1u);
+            } else if (w < ms->vis[q])
               a.scores[(rbase + q - P.row0) * a.P_cap + w] = sc;
           }
         }
@@ -407,7 +517,9 @@ __global__ void __launch_bounds__(512, 1) indexer_tc_kernel(const IdxTcParams P)
     if (n_loc <= K) {
       for (int i = tid; i < n_loc; i += kSelThreads)
         cand[i] = ((uint64_t)order_key(ssc[i]) << 32) | (uint32_t)(w0 + i);
-    } else {
+    } else if (!split_select_listed(ssc, n_loc, K, w0, shist, hist, sh,
+                                    reinterpret_cast<uint32_t*>(smem + L.a + kSelKeysOffset),
+                                    (kStages * nch * 16384 - kSelKeysOffset) / 4 / (kSelThreads / 32), cand)) {
       select_topk<kSelThreads>(
           n_loc, K, tid, [&](int i) { return order_key(ssc[i]); },
           [&](int slot, int i) { cand[slot] = ((uint64_t)order_key(ssc[i]) << 32) | (uint32_t)(w0 + i); }, hist, sh,
