@@ -177,9 +177,9 @@ NCU_TRAFFIC = {
     # took in select.cuh, which attn_tc.cu includes; it has not changed since the capture.)
     ("csa_prefill_bf16", "attention"): (_ATTN_SOURCE, "c39ebe7dad0102f834d73fa380b0cf0c41b674c81b356b8a5dadc60a1abe8bde", 1091308544),
     # ncu --set full, one launch of the CSA decode step (64 queries, pool 32768, top-2048): the fused
-    # scores + top-k kernel, dram__bytes_read.sum 535.9 MB + dram__bytes_write.sum 3.9 MB (taken after
-    # the selecting instantiation dropped the masked epilogue it never runs: 96 registers).
-    ("csa_decode_bf16", "indexer_topk"): (_INDEXER_SOURCE, "847a3d54c4c75ff5fc4cdc68d3be6faaf9fe6d0211b5efff916b864b95d08294", 539800832),
+    # scores + top-k kernel, dram__bytes_read.sum 535.8 MB + dram__bytes_write.sum 3.8 MB (taken with
+    # the split selection over per-warp lists).
+    ("csa_decode_bf16", "indexer_topk"): (_INDEXER_SOURCE, "10a99b0b9836b53ff66523ba51d13f9a831cec632672ea4f7b5f1b954f4a39a2", 539641344),
     # ncu --set full, both launches of one output-projection step (o_a_proj, then o_b_proj; the
     # part is the two launches): 608.2 + 117.7 + 604.0 + 61.5 MB.  (Re-keyed when internal.h gained
     # the attention's score-row fields; nothing this kernel compiles changed.)
