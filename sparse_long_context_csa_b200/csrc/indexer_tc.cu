@@ -585,6 +585,19 @@ bool indexer_tc_supported(const IndexerArgs& a, int dtype) {
   return true;
 }
 
+// Shared memory one CTA may opt in to on the current device (cached per device).
+int indexer_smem_optin() {
+  static int per_dev[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (per_dev[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || v <= 0) return 0;
+    per_dev[dev] = v;
+  }
+  return per_dev[dev];
+}
+
 int indexer_num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -730,6 +743,9 @@ cudaError_t launch_indexer_tc_select(const IndexerArgs& a, int64_t r0, int64_t r
   P.done = reinterpret_cast<int*>(a.scores);
   P.cand = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(a.scores) + done_bytes);
   const IdxSmem L = idx_smem_layout(a.cI, P.Npad, P.tiles_per_split * kTileE);
+  // the kept scores and their histogram take 80 KB more shared memory than the score kernel;
+  // a device that cannot give a CTA that much runs the two kernels instead
+  if ((int64_t)L.total > indexer_smem_optin()) return cudaErrorNotSupported;
   cudaError_t e = cudaMemsetAsync(P.done, 0, (size_t)rows * sizeof(int), st);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(indexer_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
