@@ -1,5 +1,6 @@
 """Host logic of bench.py that needs no GPU: the algorithmic work per part, the unit of each
-workload and whether its steps are timed with L2 flushed."""
+workload, whether its steps are timed with L2 flushed, and the source hashes that tie each
+recorded ncu DRAM figure to the kernel it was captured from."""
 from __future__ import annotations
 
 import os
@@ -87,3 +88,43 @@ def test_step_inputs_are_activations_that_exist():
     for w in synth.WORKLOADS.values():
         keys = set(harness.step_input_keys(w))
         assert not keys & {"bias", "biasI", "sink", "pool", "poolI", "win"}
+
+
+def _local_includes(name: str) -> set[str]:
+    """The csrc headers a source file includes, followed through the headers themselves."""
+    import re
+    csrc = os.path.join(ROOT, "sparse_long_context_csa_b200", "csrc")
+    seen, todo = set(), [name]
+    while todo:
+        text = open(os.path.join(csrc, todo.pop())).read()
+        for inc in re.findall(r'^#include "([^"]+)"', text, flags=re.M):
+            if inc not in seen and os.path.exists(os.path.join(csrc, inc)):
+                seen.add(inc)
+                todo.append(inc)
+    return seen
+
+
+def test_recorded_traffic_hashes_cover_each_kernel_and_its_headers():
+    """A recorded ncu DRAM figure is tied to the SHA-256 of the kernel's source: its file up to
+    the end marker, plus every csrc header the file includes.  The end marker must exist (else
+    the figure would silently never apply), and no included header may be left out of the
+    hash (else a change there would keep reporting the old figure)."""
+    for (workload, part), (segments, sha, traffic) in bench.NCU_TRAFFIC.items():
+        names = [n for n, _ in segments]
+        main, end = segments[0]
+        assert end is not None and end in open(os.path.join(
+            ROOT, "sparse_long_context_csa_b200", "csrc", main)).read(), (workload, part, "end marker")
+        missing = _local_includes(main) - set(names)
+        assert not missing, f"{workload}/{part}: headers outside the hash: {sorted(missing)}"
+        assert bench.kernel_source_sha(segments) is not None
+        assert traffic > 0 and len(sha) == 64
+
+
+def test_a_changed_kernel_reports_no_traffic(monkeypatch):
+    rec = dict(bench.NCU_TRAFFIC)
+    key = next(iter(rec))
+    segments, sha, traffic = rec[key]
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (segments, "0" * 64, traffic))
+    assert bench.ncu_traffic(*key) is None
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (segments, bench.kernel_source_sha(segments), traffic))
+    assert bench.ncu_traffic(*key) == traffic
