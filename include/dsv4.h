@@ -153,9 +153,10 @@ dsv4_status dsv4_decode_append(const dsv4_params* params, int32_t c, const void*
  *   q_index [B,Sq] int32 or NULL  cache index of each query (NULL: q_index[b,s] = s)
  *   idx     [B,Sq,topk] int32   out: selected entries in ASCENDING entry order, then -1
  *   workspace, ws_bytes         >= dsv4_workspace_bytes(params)
- * With one query per sequence (Sq == 1, bf16, nI <= 16) and about a million scored entries
- * or more per call, scores and selection run in one kernel whose score rows never leave
- * shared memory ([V32] DSA item 2); the index rows are the same, bit for bit.
+ * With one query per sequence (Sq == 1, bf16, nI <= 16), about a million scored entries
+ * or more per call and a device that lets a CTA opt in to ~216 KB of shared memory (B200:
+ * 227 KB), scores and selection run in one kernel whose score rows never leave shared
+ * memory ([V32] DSA item 2); the index rows are the same, bit for bit.
  */
 dsv4_status dsv4_indexer_topk(const dsv4_params* params, const void* qI, const float* wI,
                               const void* poolI, const int32_t* q_index, int32_t* idx,
